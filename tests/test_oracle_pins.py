@@ -1,0 +1,337 @@
+"""Pins of the CPU oracle against things other than itself (CPU only).
+
+Each test ties one oracle function to a third-party codec, a brute-force search,
+a closed form or an invariant that the mathematics of RFQ fixes, so that a
+dropped term, a wrong sign or index, or a transposed operand in the oracle fails
+at least one of them.  The method is from "Activation Outliers Matter: Robust
+Recovery for Quantized Multimodal LLMs" (section 1, RFQ contribution paragraph;
+abstract); the MXFP4 element/scale rule is OCP MX v1.0 (the pages stop before
+defining it, at section 3.1).
+"""
+import math
+
+import ml_dtypes
+import numpy as np
+import pytest
+
+from block_scaled_gemm_rfq_b200 import workloads as wl
+
+F4 = ml_dtypes.float4_e2m1fn
+
+
+# --------------------------------------------------------------------------- E2M1 decode
+def test_e2m1_decode_matches_ml_dtypes(oracle):
+    third_party = np.arange(16, dtype=np.uint8).view(F4).astype(np.float64)
+    mine = np.array([oracle.e2m1_value(c) for c in range(16)])
+    np.testing.assert_array_equal(mine, third_party)
+    # sign of zero is carried by code 8
+    assert math.copysign(1.0, oracle.e2m1_value(8)) == -1.0
+
+
+def test_e2m1_decode_matches_transformers_table(oracle):
+    mx = pytest.importorskip("transformers.integrations.mxfp4")
+    mine = [oracle.e2m1_value(c) for c in range(16)]
+    assert mine == list(mx.FP4_VALUES)
+
+
+# --------------------------------------------------------------------------- E8M0 decode
+def test_e8m0_decode_matches_torch_and_ml_dtypes(oracle):
+    import torch
+    bytes_ = np.arange(256, dtype=np.uint8)
+    want_torch = torch.from_numpy(bytes_.copy()).view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    want_mld = bytes_.view(ml_dtypes.float8_e8m0fnu).astype(np.float64)
+    # dequantize a row whose every code is 2 (value 1.0): DQ = 2^(scale-127)
+    codes = np.full((256, 16), 0x22, np.uint8)          # 32 elements, all code 2
+    scales = bytes_.reshape(256, 1)
+    dq = oracle.dequantize(codes, scales)[:, 0]
+    np.testing.assert_array_equal(dq[:255], want_torch[:255])
+    np.testing.assert_array_equal(dq[:255], want_mld[:255])
+    assert math.isnan(dq[255]) and math.isnan(want_torch[255])
+
+
+# --------------------------------------------------------------------------- scale rule
+def _brute_exponent(amax: float) -> int:
+    """The unique e in [-127, 127] with 4 <= amax * 2^-e < 8, by search; -127 if amax is below range."""
+    if amax == 0.0:
+        return -127
+    for e in range(-127, 128):
+        v = math.ldexp(amax, -e)
+        if 4.0 <= v < 8.0:
+            return e
+    assert amax < math.ldexp(4.0, -127), amax
+    return -127
+
+
+def test_block_exponent_brute_force(oracle):
+    rng = np.random.default_rng(123)
+    cands = [0.0, 1.0, 4.0, 6.0, 7.999, 8.0, 2.0 ** -126, 2.0 ** -133, 2.0 ** -125,
+             2.0 ** -125 * 0.999, 3.0e38, 2.0 ** 127, np.nextafter(2.0, 0), np.nextafter(2.0, 3)]
+    cands += list(np.exp(rng.uniform(-90, 88, 2000)))
+    # every finite positive bf16 value
+    bits = np.arange(1, 0x7F80, dtype=np.uint16)
+    cands += list(wl.bf16_bits_to_f32(bits).astype(np.float64)[::7])
+    for a in cands:
+        assert oracle.block_exponent(a) == _brute_exponent(float(a)), a
+    assert oracle.block_exponent(float("inf")) == 128
+    assert oracle.block_exponent(float("nan")) == 128
+
+
+# --------------------------------------------------------------------------- element rounding
+def _all_finite_bf16():
+    bits = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = wl.bf16_bits_to_f32(bits)
+    keep = np.isfinite(vals)
+    return bits[keep], vals[keep].astype(np.float64)
+
+
+@pytest.mark.parametrize("e", [-127, -20, -1, 0, 3, 60, 125])
+def test_element_encode_exhaustive_vs_ml_dtypes(oracle, e):
+    """Every finite bf16 x that fits a block with exponent e (|x| 2^-e < 8):
+    the oracle's code equals ml_dtypes' RNE/saturating float4_e2m1fn cast of the
+    exactly scaled value."""
+    _, x = _all_finite_bf16()
+    v = np.ldexp(x, -e)                   # exact in float64
+    keep = np.abs(v) < 8.0
+    x, v = x[keep], v[keep]
+    want = v.astype(np.float32).astype(F4).view(np.uint8)
+    got = np.array([oracle.e2m1_encode(xi, e) for xi in x], dtype=np.uint8)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, (x[bad[:5]], got[bad[:5]], want[bad[:5]])
+
+
+def test_element_encode_matches_rint_formulation(oracle):
+    """Round-half-even onto the E2M1 grid written as a different algorithm: the grid
+    spacing is 0.5 below 2, 1 in [2, 4), 2 from 4; round v/spacing with numpy's
+    rint (half to even integer = even mantissa) and clamp to 6."""
+    v = np.linspace(0.0, 7.999, 40001)
+    v = np.concatenate([v, [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0, 7.0]])
+    spacing = np.where(v < 2.0, 0.5, np.where(v < 4.0, 1.0, 2.0))
+    q = np.minimum(np.rint(v / spacing) * spacing, 6.0)
+    got = np.array([oracle.e2m1_value(oracle.e2m1_encode(vi, 0)) for vi in v])
+    np.testing.assert_array_equal(got, q)
+
+
+def test_ties_and_saturation_table(oracle):
+    # midpoints go to the neighbour with mantissa bit 0; >= 6 saturates; sign kept
+    table = {0.25: 0.0, 0.75: 1.0, 1.25: 1.0, 1.75: 2.0, 2.5: 2.0, 3.5: 4.0, 5.0: 4.0,
+             6.0: 6.0, 7.0: 6.0, 7.99: 6.0, 0.2499: 0.0, 0.2501: 0.5}
+    for v, q in table.items():
+        assert oracle.e2m1_value(oracle.e2m1_encode(v, 0)) == q
+        assert oracle.e2m1_value(oracle.e2m1_encode(-v, 0)) == -q
+    assert oracle.e2m1_encode(-0.0, 0) == 0x8
+    assert oracle.e2m1_encode(-0.1, 0) == 0x8
+    assert oracle.e2m1_encode(0.0, 0) == 0x0
+
+
+# --------------------------------------------------------------------------- block quantizer
+def test_qdq_identity_on_representable_blocks(oracle):
+    """Blocks of grid values times 2^t whose amax is 4*2^t or 6*2^t are reproduced
+    exactly by DQ(Q(x)); their residual is zero, so Q(R) is all code 0, scale 0."""
+    rng = np.random.default_rng(7)
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    rows = []
+    for t in [-120, -30, -3, 0, 2, 40, 100]:
+        for top in (4.0, 6.0):
+            g = rng.choice(grid[grid <= top], 32) * rng.choice([-1.0, 1.0], 32)
+            g[rng.integers(32)] = top * rng.choice([-1.0, 1.0])
+            rows.append(np.ldexp(g, t))
+    X = np.array(rows)
+    bits = wl.f64_to_bf16_bits(X)
+    assert np.array_equal(wl.bf16_bits_to_f32(bits).astype(np.float64), X)
+    q = oracle.quantize_bf16(bits)
+    np.testing.assert_array_equal(oracle.dequantize(q["codes_x"], q["scales_x"]), X)
+    assert not (q["codes_r"] & 0x7).any()
+    assert not q["scales_r"].any()
+
+
+def _rand_heavy(rows, K, seed):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_t(3.0, (rows, K))
+    X[:, rng.choice(K, max(1, K // 50), replace=False)] *= 100.0
+    X[rng.random((rows, K)) < 0.01] *= 1e-30          # tiny values next to large ones
+    return wl.f64_to_bf16_bits(X)
+
+
+def test_residual_is_full_error_and_requantized_by_same_rule(oracle):
+    """Q(R) from the bf16 quantizer equals the plain-float64 quantizer applied to
+    R = X - DQ(Q(X)) computed here by dequantization (two code paths)."""
+    bits = _rand_heavy(64, 512, 11)
+    X = wl.bf16_bits_to_f32(bits).astype(np.float64)
+    q = oracle.quantize_bf16(bits)
+    R = X - oracle.dequantize(q["codes_x"], q["scales_x"])
+    codes_r, scales_r = oracle.quantize_f64(R)
+    np.testing.assert_array_equal(codes_r, q["codes_r"])
+    np.testing.assert_array_equal(scales_r, q["scales_r"])
+    # R is exactly representable in fp32 (the GPU keeps it in fp32)
+    np.testing.assert_array_equal(R.astype(np.float32).astype(np.float64), R)
+
+
+def test_residual_never_increases_error(oracle):
+    """Elementwise |r - DQ(Q(r))| <= |r| (0 is on the grid), hence on every block
+    ||X - DQ(QX) - DQ(QR)|| <= ||X - DQ(QX)||."""
+    bits = _rand_heavy(128, 1024, 12)
+    X = wl.bf16_bits_to_f32(bits).astype(np.float64)
+    q = oracle.quantize_bf16(bits)
+    DX = oracle.dequantize(q["codes_x"], q["scales_x"])
+    DR = oracle.dequantize(q["codes_r"], q["scales_r"])
+    R = X - DX
+    assert np.all(np.abs(R - DR) <= np.abs(R))
+    e1 = ((R) ** 2).reshape(128, -1, 32).sum(-1)
+    e2 = ((R - DR) ** 2).reshape(128, -1, 32).sum(-1)
+    assert np.all(e2 <= e1)
+    assert e2.sum() < 0.1 * e1.sum()          # the residual path recovers most of the error
+
+
+def test_residual_scale_invariant(oracle):
+    """|r| < 2^(e_X + 1) so the residual scale byte is <= max(byte_X - 2, 0)."""
+    bits = _rand_heavy(128, 1024, 13)
+    q = oracle.quantize_bf16(bits)
+    sx = q["scales_x"].astype(int)
+    sr = q["scales_r"].astype(int)
+    assert np.all(sr <= np.maximum(sx - 2, 0))
+
+
+def test_all_zero_and_signed_zero_blocks(oracle):
+    bits = np.zeros((2, 64), np.uint16)
+    bits[1, :] = 0x8000                                    # -0.0
+    q = oracle.quantize_bf16(bits)
+    assert not q["scales_x"].any() and not q["scales_r"].any()
+    assert not q["codes_x"][0].any()
+    assert np.all(q["codes_x"][1] == 0x88)
+    # IEEE: r = (-0) - (-0) = +0, so the residual of a -0 block is +0
+    assert not q["codes_r"][1].any()
+
+
+def test_nonfinite_block_gets_nan_scale(oracle):
+    bits = wl.random_matrix(2, 64, seed=3)
+    bits[0, 5] = 0x7F80          # +inf in block 0 of row 0
+    bits[1, 40] = 0x7FC0         # NaN in block 1 of row 1
+    q = oracle.quantize_bf16(bits)
+    assert q["scales_x"][0, 0] == 0xFF and q["scales_r"][0, 0] == 0xFF
+    assert q["scales_x"][1, 1] == 0xFF and q["scales_r"][1, 1] == 0xFF
+    assert q["scales_x"][0, 1] != 0xFF and q["scales_x"][1, 0] != 0xFF
+
+
+def test_subnormal_blocks(oracle):
+    """bf16 subnormals: the exponent clamps to -127 (byte 0) and nothing is flushed."""
+    bits = np.zeros((1, 32), np.uint16)
+    bits[0, :] = np.arange(1, 33, dtype=np.uint16)        # 1..32 x 2^-133
+    q = oracle.quantize_bf16(bits)
+    assert q["scales_x"][0, 0] == 0
+    X = wl.bf16_bits_to_f32(bits).astype(np.float64)
+    dx = oracle.dequantize(q["codes_x"], q["scales_x"])
+    # scaled values are 2^-6 .. 2^-1: 2^127 * 32 * 2^-133 = 0.5, the largest becomes code 1
+    assert dx[0, -1] == X[0, -1]
+    assert q["codes_x"][0, -1] >> 4 == 1
+
+
+# --------------------------------------------------------------------------- reference GEMM
+def test_gemm_loops_match_blas_and_closed_forms(oracle):
+    rng = np.random.default_rng(5)
+    A = rng.standard_normal((37, 96))
+    B = rng.standard_normal((23, 96))
+    Y, absY = oracle.gemm_loops(A, B)
+    Yb, absYb = oracle.gemm_blas(A, B)
+    np.testing.assert_allclose(Y, Yb, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(absY, absYb, rtol=1e-14)
+    # closed form: B = identity rows picks columns of A
+    I = np.eye(96)[:23]
+    Yi, _ = oracle.gemm_loops(A, I)
+    np.testing.assert_array_equal(Yi, A[:, :23])
+    # transposition check: swapping operands transposes Y
+    Yt, _ = oracle.gemm_loops(B, A)
+    np.testing.assert_array_equal(Yt, Y.T)
+
+
+def test_rfq_gemm_is_sum_of_two_terms(oracle):
+    """Y = DQ(QX).DQ(QW)^T + DQ(QR).DQ(QW)^T, and with RFQ off the first term alone."""
+    w = wl.tiny(0)
+    Y, S, _ = oracle.rfq_linear(w.x_bits, w.w_bits, residual=True)
+    Yoff, Soff, _ = oracle.rfq_linear(w.x_bits, w.w_bits, residual=False)
+    qa = oracle.quantize_bf16(w.x_bits)
+    qw = oracle.quantize_bf16(w.w_bits, residual=False)
+    DX = oracle.dequantize(qa["codes_x"], qa["scales_x"])
+    DR = oracle.dequantize(qa["codes_r"], qa["scales_r"])
+    DW = oracle.dequantize(qw["codes_x"], qw["scales_x"])
+    np.testing.assert_allclose(Y, DX @ DW.T + DR @ DW.T, rtol=0, atol=1e-9 * S)
+    np.testing.assert_allclose(Yoff, DX @ DW.T, rtol=0, atol=1e-9 * Soff)
+    assert S >= Soff
+
+
+def test_rfq_recovers_activation_fidelity(oracle):
+    """The paper's central claim on synthetic heavy-tailed inputs: adding the
+    residual term brings Y much closer to the unquantized product X.W^T."""
+    w = wl.tiny(0)
+    X = wl.bf16_bits_to_f32(w.x_bits).astype(np.float64)
+    W = wl.bf16_bits_to_f32(w.w_bits).astype(np.float64)
+    exact = X @ W.T
+    Y, _, _ = oracle.rfq_linear(w.x_bits, w.w_bits, residual=True)
+    Yoff, _, _ = oracle.rfq_linear(w.x_bits, w.w_bits, residual=False)
+    assert np.linalg.norm(Y - exact) < 0.8 * np.linalg.norm(Yoff - exact)
+    # activation error alone (weights held at DQ(QW)): the residual path removes most of it
+    qw = oracle.quantize_bf16(w.w_bits, residual=False)
+    act_only = X @ oracle.dequantize(qw["codes_x"], qw["scales_x"]).T
+    assert np.linalg.norm(Y - act_only) < 0.3 * np.linalg.norm(Yoff - act_only)
+
+
+# --------------------------------------------------------------------------- scale layout
+def test_mma_scale_layout_known_offsets_and_bijection(oracle):
+    Kb = 10                                   # Kb_pad = 12 -> 3 atoms per 128-row tile
+    assert oracle.mma_scale_offset(0, 0, Kb) == 0
+    assert oracle.mma_scale_offset(0, 1, Kb) == 1
+    assert oracle.mma_scale_offset(0, 3, Kb) == 3
+    assert oracle.mma_scale_offset(1, 0, Kb) == 16
+    assert oracle.mma_scale_offset(31, 0, Kb) == 31 * 16
+    assert oracle.mma_scale_offset(32, 0, Kb) == 4
+    assert oracle.mma_scale_offset(96, 2, Kb) == 14
+    assert oracle.mma_scale_offset(0, 4, Kb) == 512
+    assert oracle.mma_scale_offset(128, 0, Kb) == 3 * 512
+    rows = 200
+    offs = {oracle.mma_scale_offset(r, c, Kb) for r in range(256) for c in range(12)}
+    assert offs == set(range(256 * 12))
+    plain = np.random.default_rng(0).integers(1, 255, (rows, Kb), dtype=np.uint8)
+    lay = oracle.scales_to_mma_layout(plain)
+    assert lay.size == 256 * 12
+    back = np.array([[lay[oracle.mma_scale_offset(r, c, Kb)] for c in range(Kb)] for r in range(rows)])
+    np.testing.assert_array_equal(back, plain)
+    assert int(lay.astype(np.int64).sum()) == int(plain.astype(np.int64).sum())   # padding is 0
+
+
+def test_workload_generators_are_seeded():
+    a = wl.tiny(0)
+    b = wl.tiny(0)
+    c = wl.tiny(1)
+    assert np.array_equal(a.x_bits, b.x_bits) and np.array_equal(a.w_bits, b.w_bits)
+    assert not np.array_equal(a.x_bits, c.x_bits)
+    X = wl.bf16_bits_to_f32(a.x_bits)
+    assert np.abs(X[:, 7]).mean() > 20 and np.abs(X[:, 8]).mean() < 2
+
+
+# --------------------------------------------------------------------------- regression + isolation
+def test_oracle_matches_committed_golden_digest(oracle):
+    """tests/golden/tiny_oracle_digest.json was written by tests/golden/make_golden.py
+    (oracle only); a change of the oracle's arithmetic must regenerate it knowingly."""
+    import json
+    import os
+    import sys
+    sys.path.insert(0, os.path.join(os.path.dirname(__file__), "golden"))
+    import make_golden
+    with open(os.path.join(os.path.dirname(__file__), "golden", "tiny_oracle_digest.json")) as f:
+        want = json.load(f)
+    got = make_golden.compute()
+    for k, v in want.items():
+        if isinstance(v, float):
+            assert got[k] == pytest.approx(v, rel=1e-12, abs=1e-300), k
+        else:
+            assert got[k] == v, k
+
+
+def test_oracle_shares_nothing_with_cuda_path():
+    import os
+    import re
+    here = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for name in os.listdir(os.path.join(here, "oracle")):
+        if name.endswith((".py", ".c", ".h")):
+            src = open(os.path.join(here, "oracle", name)).read()
+            assert not re.search(r"^\s*(from|import)\s+block_scaled_gemm_rfq_b200", src, re.M), name
+            assert "#include \"rfq.h\"" not in src and "csrc" not in src, name
