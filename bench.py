@@ -1,0 +1,474 @@
+"""Benchmark of the RFQ MXFP4 W4A4 linear layer on B200 (one JSON line on rank 0).
+
+A step is one pass of the whole hot path on the LLM FFN up-projection workload
+(X bf16 4096 x 4096 with outlier channels and spikes, W bf16 12288 x 4096, Y bf16):
+  1. rfq_quantize_weight   W -> Q(W)                       (kernel 1, no residual)
+  2. rfq_quantize_mxfp4    X -> Q(X), Q(R), R = X - DQ(Q(X)) (kernel 1, fused)
+  3. rfq_gemm              Y = DQ(QX) DQ(QW)^T + DQ(QR) DQ(QW)^T (kernel 2, tcgen05)
+Inputs are resident in HBM; L2 is flushed (256 MiB write) between timed steps,
+outside the per-step CUDA events.  ``value`` is executed MMA TFLOP/s over the
+whole step (4*M*N*K per step: the residual doubles K on the tensor pipe).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--all-configs]
+
+N > 1 runs under torchrun: every rank runs its own replica of the step (the
+layer has no exchange step; weak scaling), time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense MXFP4 : bf16 tensor throughput on B200
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = self._handle(pynvml, device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    @staticmethod
+    def _handle(pynvml, device_index):
+        # NVML enumerates every GPU of the machine; find the one torch uses by UUID
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(device_index)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nvml.nvmlDeviceGetClockInfo(self._h, self._nvml.NVML_CLOCK_SM))
+                r = self._nvml.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nvml:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._nvml:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        from datetime import timedelta
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+        return dist.get_rank(), world, local
+    return 0, 1, 0
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- the CUDA path
+def to_device_bf16(bits):
+    import numpy as np
+    import torch
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+
+
+class RfqStep:
+    """Buffers and launches of one step (all through the C ABI binding)."""
+
+    def __init__(self, rfq, x, w, residual=True, out_dtype=None):
+        import torch
+        self.rfq, self.x, self.w, self.residual = rfq, x, w, residual
+        self.M, self.K = x.shape
+        self.N = w.shape[0]
+        dev = x.device
+        u8 = lambda n: torch.empty(max(n, 1), dtype=torch.uint8, device=dev)
+        self.qw_c, self.qw_s = u8(rfq.codes_bytes(self.N, self.K)), u8(rfq.scales_bytes(self.N, self.K))
+        self.qx_c, self.qx_s = u8(rfq.codes_bytes(self.M, self.K)), u8(rfq.scales_bytes(self.M, self.K))
+        self.qr_c = u8(rfq.codes_bytes(self.M, self.K)) if residual else None
+        self.qr_s = u8(rfq.scales_bytes(self.M, self.K)) if residual else None
+        self.y = torch.empty((self.M, self.N), dtype=out_dtype or torch.bfloat16, device=dev)
+
+    def quantize_w(self):
+        self.rfq.quantize_weight(self.w, self.qw_c, self.qw_s)
+
+    def quantize_x(self):
+        self.rfq.quantize_mxfp4(self.x, self.qx_c, self.qx_s, self.qr_c, self.qr_s)
+
+    def gemm(self):
+        self.rfq.gemm(self.qx_c, self.qx_s, self.qr_c, self.qr_s, self.qw_c, self.qw_s, self.M, self.N, self.K,
+                      self.y)
+
+    def run(self):
+        self.quantize_w()
+        self.quantize_x()
+        self.gemm()
+
+
+def time_phases(step: RfqStep, steps: int, warmup: int, flush, world: int):
+    """Per-step CUDA events around each kernel; L2 flushed between steps."""
+    import torch
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush()
+        e = ev[i]
+        e[0].record()
+        step.quantize_w()
+        e[1].record()
+        step.quantize_x()
+        e[2].record()
+        step.gemm()
+        e[3].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    qw = [e[0].elapsed_time(e[1]) for e in ev]
+    qx = [e[1].elapsed_time(e[2]) for e in ev]
+    gm = [e[2].elapsed_time(e[3]) for e in ev]
+    tot = [e[0].elapsed_time(e[3]) for e in ev]
+    return {"quantize_w_ms": qw, "quantize_x_ms": qx, "gemm_ms": gm, "step_ms": tot}
+
+
+def time_kernel(fn, iters, flush):
+    import torch
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    out = []
+    for _ in range(iters):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        out.append((a, b))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in out]
+
+
+def quantize_bytes(M, K, residual):
+    """Algorithmic HBM bytes of the fused quantizer: read X once (2 B/elem), write codes
+    (0.5 B/elem) and scales (1 B per 32 elements) per output."""
+    outs = 2 if residual else 1
+    return M * K * 2 + outs * (M * K // 2 + M * K // 32)
+
+
+def run_cuda(args, rank, world, local):
+    import numpy as np
+    import torch
+
+    import block_scaled_gemm_rfq_b200 as rfq
+    from block_scaled_gemm_rfq_b200 import workloads as wl
+
+    rfq.load_library()
+    peaks = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    hbm_peak = peaks["hbm_gbs"]
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = lambda: flush_buf.zero_()
+
+    wk = wl.ffn_up(seed=rank)
+    M, K, N = wk.M, wk.K, wk.N
+    x, w = to_device_bf16(wk.x_bits), to_device_bf16(wk.w_bits)
+    step = RfqStep(rfq, x, w, residual=True)
+    flops = 4.0 * M * N * K
+
+    with ClockSampler(local) as clk:
+        ph = time_phases(step, args.steps, args.warmup, flush, world)
+    rfq.check_device_error()
+    step_ms_total = sum(ph["step_ms"])
+    step_ms_max = max_over_ranks(step_ms_total, world)
+    ms_per_step = step_ms_max / args.steps
+    value = world * flops * args.steps / (step_ms_max * 1e-3) / 1e12
+
+    gemm_ms = statistics.mean(ph["gemm_ms"])
+    qx_ms = statistics.mean(ph["quantize_x_ms"])
+    qw_ms = statistics.mean(ph["quantize_w_ms"])
+    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
+
+    extra = {}
+    # RFQ off (plain MXFP4): the overhead the pages call negligible
+    off = RfqStep(rfq, x, w, residual=False)
+    off.quantize_w()
+    off.quantize_x()
+    t_off = time_kernel(off.gemm, max(10, args.steps // 2), flush)
+    t_on = time_kernel(step.gemm, max(10, args.steps // 2), flush)
+    extra["rfq_off"] = {"gemm_ms": statistics.mean(t_off), "gemm_ms_rfq": statistics.mean(t_on),
+                        "gemm_overhead": statistics.mean(t_on) / statistics.mean(t_off),
+                        "tflops_executed": 2.0 * M * N * K / (statistics.mean(t_off) * 1e-3) / 1e12}
+    del off
+
+    # quantize-only bandwidth workload (8192 x 4096, heavy-tailed)
+    qb = wl.quantize_bandwidth(seed=rank)
+    xq = to_device_bf16(qb.x_bits)
+    qstep = RfqStep(rfq, xq, w[:8], residual=True)
+    tq = time_kernel(qstep.quantize_x, max(20, args.steps), flush)
+    qbytes = quantize_bytes(qb.M, qb.K, True)
+    q_gbs = qbytes / (statistics.mean(tq) * 1e-3) / 1e9
+    extra["quantize_bandwidth"] = {"workload": qb.name, "ms": statistics.mean(tq), "ms_min": min(tq),
+                                   "bytes": qbytes, "gbs": q_gbs, "frac_hbm": q_gbs / hbm_peak}
+    del qstep, xq
+
+    if args.all_configs:
+        dk = wl.dit_ffn(seed=rank)
+        xd, wd = to_device_bf16(dk.x_bits), to_device_bf16(dk.w_bits)
+        for res in (True, False):
+            s2 = RfqStep(rfq, xd, wd, residual=res)
+            s2.quantize_w()
+            s2.quantize_x()
+            t = time_kernel(s2.gemm, 10, flush)
+            f = (4.0 if res else 2.0) * dk.M * dk.N * dk.K
+            extra[f"dit_ffn_gemm_{'rfq' if res else 'off'}"] = {
+                "ms": statistics.mean(t), "tflops_executed": f / (statistics.mean(t) * 1e-3) / 1e12,
+                "frac_fp4_peak": f / (statistics.mean(t) * 1e-3) / 1e12 / fp4_peak}
+            del s2
+        del xd, wd
+        sweep = {}
+        for Ms in wl.SWEEP_M:
+            sk = wl.m_sweep(Ms, seed=rank)
+            xs, ws = to_device_bf16(sk.x_bits), to_device_bf16(sk.w_bits)
+            row = {}
+            for res in (True, False):
+                qws = rfq.quantize_weight_alloc(ws)
+                y = torch.empty((Ms, sk.N), dtype=torch.bfloat16, device="cuda")
+                wsb = torch.empty(rfq.linear_workspace_bytes(Ms, sk.K, res), dtype=torch.uint8, device="cuda")
+                t = time_kernel(lambda: rfq.linear(xs, qws.codes, qws.scales, sk.N, y, wsb, res), 20, flush)
+                row["rfq" if res else "off"] = {"us": 1e3 * statistics.mean(t),
+                                                "tflops_useful": 2.0 * Ms * sk.N * sk.K / (statistics.mean(t) * 1e-3) / 1e12}
+            sweep[str(Ms)] = row
+        extra["m_sweep_rfq_linear"] = sweep
+
+    # end to end through the public API with host buffers: pinned X, W in; Y out
+    xh = torch.from_numpy(wk.x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    wh = torch.from_numpy(wk.w_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(5, args.steps // 4)
+
+    def e2e_once():
+        x.copy_(xh, non_blocking=True)
+        w.copy_(wh, non_blocking=True)
+        step.run()
+        yh.copy_(step.y, non_blocking=True)
+
+    for _ in range(2):
+        e2e_once()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(e2e_steps):
+        e2e_once()
+    b.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b), world) / e2e_steps
+    rfq.check_device_error()
+
+    result = {
+        "metric": "RFQ W4A4 GEMM TFLOPS (% MXFP4 peak); fused RFQ quantize GB/s (% HBM)",
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "mxfp4 (e2m1 x e2m1, e8m0 scales), fp32 accumulate, bf16 out",
+        "data": "synthetic (seeded numpy: N(0,1) + 0.5% outlier channels x50 + 0.01% spikes x500; W N(0,0.02))",
+        "config": {"workload": wk.name, "M": M, "K": K, "N": N, "rfq": True, "y": "bf16",
+                   "step": "rfq_quantize_weight + rfq_quantize_mxfp4 (X, residual) + rfq_gemm",
+                   "l2": "flushed between steps (256 MiB write, outside the step events)",
+                   "parallelism": f"replicas x{world}"},
+        "gemm": {"ms": gemm_ms, "tflops_executed": gemm_tflops, "tflops_useful": gemm_tflops / 2,
+                 "frac_fp4_peak": gemm_tflops / fp4_peak},
+        "quantize_x": {"ms": qx_ms, "gbs": quantize_bytes(M, K, True) / (qx_ms * 1e-3) / 1e9},
+        "quantize_w": {"ms": qw_ms, "gbs": quantize_bytes(N, K, False) / (qw_ms * 1e-3) / 1e9},
+        "roofline": {"bound": "tensor", "kernel": "rfq_gemm_kernel<residual, bf16>", "achieved": gemm_tflops,
+                     "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
+                     "peak_basis": f"{peaks['source']} bf16_tflops {peaks['bf16_tflops']} x {FP4_OVER_BF16} "
+                                   "(nominal MXFP4:bf16 ratio), burst",
+                     "traffic": None},
+        "roofline_quantize": {"bound": "hbm", "kernel": "rfq_quantize_kernel<residual>",
+                              "achieved": extra["quantize_bandwidth"]["gbs"], "peak": hbm_peak, "unit": "GB/s",
+                              "frac": extra["quantize_bandwidth"]["gbs"] / hbm_peak,
+                              "peak_basis": f"{peaks['source']} hbm_gbs", "traffic": None},
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": int(xh.numel() * 2 + wh.numel() * 2),
+                "d2h_bytes_per_step": int(yh.numel() * 2)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+        "gpu": torch.cuda.get_device_name(),
+    }
+    result.update(extra)
+    if rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wk, args.cpu_seconds)
+    return result
+
+
+# ----------------------------------------------------------------------------- the oracle on the host cores
+def cpu_baseline(wk, budget_s: float):
+    """The CPU oracle, as it stands, on a bounded sample of the same step, scaled to the
+    whole step: quantize n_w rows of W, m rows of X (with residual), and the float64
+    reference GEMM of those m rows against n_w columns; extrapolated by rows."""
+    import numpy as np
+
+    import oracle
+    oracle.build()
+    M, K, N = wk.M, wk.K, wk.N
+    m = 32
+    nw = 1024
+    t0 = time.perf_counter()
+    qw = oracle.quantize_bf16(wk.w_bits[:nw], residual=False)
+    t_qw = (time.perf_counter() - t0) * (N / nw)
+    t0 = time.perf_counter()
+    qa = oracle.quantize_bf16(wk.x_bits[:m], residual=True)
+    t_qx = (time.perf_counter() - t0) * (M / m)
+    A, B = oracle.rfq_operands(qa, qw, True)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.gemm_blas(A, B)
+        reps += 1
+        if time.perf_counter() - t0 > min(5.0, budget_s / 3):
+            break
+    t_gemm = (time.perf_counter() - t0) / reps * (M / m) * (N / nw)
+    total = t_qw + t_qx + t_gemm
+    cores = len(os.sched_getaffinity(0))
+    return {"value": 4.0 * M * N * K / total / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "seconds_per_step_extrapolated": total,
+            "parts_s": {"quantize_w": t_qw, "quantize_x": t_qx, "gemm_f64": t_gemm},
+            "sample": f"oracle quantize of W rows [0,{nw}) and X rows [0,{m}) (C, 1 thread), float64 "
+                      f"numpy matmul of those X rows x W rows (BLAS, up to {cores} threads), "
+                      f"each scaled by rows to the full {M}x{K}x{N} step"}
+
+
+def run_reference(args):
+    """--impl reference: the oracle, timed on the host cores on this workload's bounded
+    samples, reported in the same metric/unit."""
+    from block_scaled_gemm_rfq_b200 import workloads as wl
+    wk = wl.ffn_up(seed=0)
+    samples = []
+    for _ in range(args.warmup):
+        cpu_baseline(wk, args.cpu_seconds)
+    for _ in range(args.steps):
+        samples.append(cpu_baseline(wk, args.cpu_seconds))
+    v = statistics.mean(s["value"] for s in samples)
+    cb = dict(samples[-1])
+    cb["value"] = v
+    return {
+        "impl": "reference",
+        "metric": "RFQ W4A4 GEMM TFLOPS (% MXFP4 peak); fused RFQ quantize GB/s (% HBM)",
+        "value": v, "unit": "TFLOP/s", "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(s["seconds_per_step_extrapolated"] for s in samples),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+        "data": "synthetic (same seeded generator as the CUDA arm)",
+        "config": {"workload": wk.name, "M": wk.M, "K": wk.K, "N": wk.N, "rfq": True, "y": "f64"},
+        "cpu_baseline": cb,
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--all-configs", action="store_true", help="also time the DiT FFN GEMM and the M sweep")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        print(json.dumps(run_reference(args)))
+        return
+
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        res = run_cuda(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(res))
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,213 @@
+"""B200 (sm_100a) Residual Fallback Quantization: MXFP4 W4A4 linear layers.
+
+Python binding of the C ABI in include/rfq.h (``librfq.so``, built in-tree by
+``block_scaled_gemm_rfq_b200.build``).  This module only marshals arguments:
+every step of the path (quantization, residual, requantization, GEMM) runs in the
+library's CUDA kernels.  PyTorch is used for device memory and streams.  There is
+no CPU fallback: if the library is missing, every call raises.
+
+Method: "Activation Outliers Matter: Robust Recovery for Quantized Multimodal
+LLMs" (arXiv 2608.26581), section 1 (RFQ): Y = (DQ(QX) + DQ(QR)) DQ(QW)^T with
+R = X - DQ(QX) requantized by the same MXFP4 rule.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = [
+    "RFQError", "load_library", "library_path", "codes_bytes", "scales_bytes", "linear_workspace_bytes",
+    "quantize_mxfp4", "quantize_weight", "gemm", "linear", "check_device_error", "debug_skip_next_fill",
+    "QuantizedTensor", "quantize_mxfp4_alloc", "quantize_weight_alloc", "gemm_alloc", "linear_alloc",
+    "EXPORTED_SYMBOLS", "OUT_F32", "OUT_BF16",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "librfq.so")
+_lock = threading.Lock()
+_lib = None
+
+OUT_F32 = 0
+OUT_BF16 = 1
+
+STATUS = {0: "RFQ_OK", 1: "RFQ_ERR_INVALID_ARG", 2: "RFQ_ERR_UNSUPPORTED_SHAPE", 3: "RFQ_ERR_MISALIGNED",
+          4: "RFQ_ERR_UNSUPPORTED_DEVICE", 5: "RFQ_ERR_CUDA", 6: "RFQ_ERR_TIMEOUT", 7: "RFQ_ERR_WORKSPACE"}
+
+# Every function include/rfq.h declares (checked against the built library by the CPU tests).
+EXPORTED_SYMBOLS = (
+    "rfq_status_string", "rfq_codes_bytes", "rfq_scales_bytes", "rfq_quantize_mxfp4", "rfq_quantize_weight",
+    "rfq_gemm", "rfq_linear_workspace_bytes", "rfq_linear", "rfq_check_device_error", "rfq_debug_skip_next_fill",
+)
+
+
+class RFQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load librfq.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(f"CUDA library {_LIB_PATH} is missing; build it with "
+                                   "`python -m block_scaled_gemm_rfq_b200.build`")
+            lib = ctypes.CDLL(_LIB_PATH)
+            P, I64, SZ, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+            sig = {
+                "rfq_status_string": (ctypes.c_char_p, [I]),
+                "rfq_codes_bytes": (SZ, [I64, I64]),
+                "rfq_scales_bytes": (SZ, [I64, I64]),
+                "rfq_quantize_mxfp4": (I, [P, I64, I64, P, P, P, P, P]),
+                "rfq_quantize_weight": (I, [P, I64, I64, P, P, P]),
+                "rfq_gemm": (I, [P, P, P, P, P, P, I64, I64, I64, P, I, P]),
+                "rfq_linear_workspace_bytes": (SZ, [I64, I64, I]),
+                "rfq_linear": (I, [P, I64, I64, P, P, I64, P, I, I, P, SZ, P]),
+                "rfq_check_device_error": (I, [P, ctypes.POINTER(ctypes.c_int)]),
+                "rfq_debug_skip_next_fill": (I, [I]),
+            }
+            for name, (res, args) in sig.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise RFQError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+# ----------------------------------------------------------------------------- sizes
+def codes_bytes(rows: int, K: int) -> int:
+    return int(load_library().rfq_codes_bytes(rows, K))
+
+
+def scales_bytes(rows: int, K: int) -> int:
+    return int(load_library().rfq_scales_bytes(rows, K))
+
+
+def linear_workspace_bytes(M: int, K: int, use_residual: bool = True) -> int:
+    return int(load_library().rfq_linear_workspace_bytes(M, K, int(bool(use_residual))))
+
+
+# ----------------------------------------------------------------------------- raw calls (caller-owned buffers)
+def quantize_mxfp4(x, qx_codes, qx_scales, qr_codes=None, qr_scales=None, stream=None):
+    """rfq_quantize_mxfp4 on torch tensors: x [M, K] bf16 (CUDA), outputs uint8 buffers."""
+    M, K = x.shape
+    _check(load_library().rfq_quantize_mxfp4(_ptr(x), M, K, _ptr(qx_codes), _ptr(qx_scales), _ptr(qr_codes),
+                                             _ptr(qr_scales), _stream(stream)), "rfq_quantize_mxfp4")
+
+
+def quantize_weight(w, qw_codes, qw_scales, stream=None):
+    N, K = w.shape
+    _check(load_library().rfq_quantize_weight(_ptr(w), N, K, _ptr(qw_codes), _ptr(qw_scales), _stream(stream)),
+           "rfq_quantize_weight")
+
+
+def gemm(qx_codes, qx_scales, qr_codes, qr_scales, qw_codes, qw_scales, M, N, K, y, stream=None):
+    """rfq_gemm; y's dtype (float32 or bfloat16) selects the output type."""
+    import torch
+    y_type = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
+    _check(load_library().rfq_gemm(_ptr(qx_codes), _ptr(qx_scales), _ptr(qr_codes), _ptr(qr_scales),
+                                   _ptr(qw_codes), _ptr(qw_scales), M, N, K, _ptr(y), y_type, _stream(stream)),
+           "rfq_gemm")
+
+
+def linear(x, qw_codes, qw_scales, N, y, workspace, use_residual=True, stream=None):
+    import torch
+    M, K = x.shape
+    y_type = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
+    _check(load_library().rfq_linear(_ptr(x), M, K, _ptr(qw_codes), _ptr(qw_scales), N, _ptr(y), y_type,
+                                     int(bool(use_residual)), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "rfq_linear")
+
+
+def check_device_error(stream=None):
+    """Synchronize and report a bounded-wait timeout inside a kernel (raises RFQError)."""
+    detail = ctypes.c_int(0)
+    st = load_library().rfq_check_device_error(_stream(stream), ctypes.byref(detail))
+    if st != 0:
+        err = RFQError(st, f"rfq_check_device_error (detail {detail.value})")
+        err.detail = detail.value
+        raise err
+    return 0
+
+
+def debug_skip_next_fill(fill_index: int):
+    load_library().rfq_debug_skip_next_fill(int(fill_index))
+
+
+# ----------------------------------------------------------------------------- allocating conveniences
+class QuantizedTensor:
+    """Codes and MMA-layout scales of an MXFP4 matrix [rows, K] (plus Q(R) when present)."""
+
+    def __init__(self, rows, K, codes, scales, r_codes=None, r_scales=None):
+        self.rows, self.K = rows, K
+        self.codes, self.scales = codes, scales
+        self.r_codes, self.r_scales = r_codes, r_scales
+
+    @property
+    def has_residual(self):
+        return self.r_codes is not None
+
+
+def _empty_u8(n, device):
+    import torch
+    # over-allocate by nothing; torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(int(n), 1), dtype=torch.uint8, device=device)
+
+
+def quantize_mxfp4_alloc(x, residual=True, stream=None) -> QuantizedTensor:
+    M, K = x.shape
+    cb, sb = codes_bytes(M, K), scales_bytes(M, K)
+    q = QuantizedTensor(M, K, _empty_u8(cb, x.device), _empty_u8(sb, x.device),
+                        _empty_u8(cb, x.device) if residual else None, _empty_u8(sb, x.device) if residual else None)
+    quantize_mxfp4(x, q.codes, q.scales, q.r_codes, q.r_scales, stream)
+    return q
+
+
+def quantize_weight_alloc(w, stream=None) -> QuantizedTensor:
+    N, K = w.shape
+    q = QuantizedTensor(N, K, _empty_u8(codes_bytes(N, K), w.device), _empty_u8(scales_bytes(N, K), w.device))
+    quantize_weight(w, q.codes, q.scales, stream)
+    return q
+
+
+def gemm_alloc(qa: QuantizedTensor, qw: QuantizedTensor, out_dtype=None, use_residual=True, stream=None):
+    import torch
+    out_dtype = out_dtype or torch.bfloat16
+    y = torch.empty((qa.rows, qw.rows), dtype=out_dtype, device=qa.codes.device)
+    res = use_residual and qa.has_residual
+    gemm(qa.codes, qa.scales, qa.r_codes if res else None, qa.r_scales if res else None, qw.codes, qw.scales,
+         qa.rows, qw.rows, qa.K, y, stream)
+    return y
+
+
+def linear_alloc(x, qw: QuantizedTensor, out_dtype=None, use_residual=True, stream=None):
+    import torch
+    M, K = x.shape
+    out_dtype = out_dtype or torch.bfloat16
+    y = torch.empty((M, qw.rows), dtype=out_dtype, device=x.device)
+    ws = _empty_u8(linear_workspace_bytes(M, K, use_residual), x.device)
+    linear(x, qw.codes, qw.scales, qw.rows, y, ws, use_residual, stream)
+    return y

@@ -1,0 +1,26 @@
+// rfq_internal.h -- launchers shared between the kernels' .cu files and the C ABI.
+// Arguments are validated by the C ABI (rfq_api.cu) before these are called.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace rfq {
+
+// Kernel 1: fused quantizer.  qr_codes == nullptr selects plain MXFP4.
+cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, void* qx_codes, void* qx_scales, void* qr_codes,
+                            void* qr_scales, int num_sms, cudaStream_t stream);
+
+// Kernel 2: RFQ GEMM.  qr_codes == nullptr selects the plain MXFP4 GEMM.
+// `encode_tiled` is the driver's cuTensorMapEncodeTiled.  `skip_fill` >= 0 makes
+// the producer of CTA 0 skip that stage fill (fault injection for the bounded
+// waits; -1 in normal use).
+cudaError_t launch_gemm(const void* qx_codes, const void* qx_scales, const void* qr_codes, const void* qr_scales,
+                        const void* qw_codes, const void* qw_scales, int64_t M, int64_t N, int64_t K, void* y,
+                        bool y_bf16, int num_sms, void* encode_tiled, int skip_fill, cudaStream_t stream);
+
+// Read and clear the device error word of the current device.
+cudaError_t read_and_clear_device_error(unsigned int* value);
+
+}  // namespace rfq

@@ -29,9 +29,9 @@ import numpy as np
 
 def f64_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """float64 -> float32 (RNE) -> bf16 (RNE) bit patterns as uint16.  Finite inputs only."""
-    f32 = np.ascontiguousarray(a, dtype=np.float32)
-    u = f32.view(np.uint32).astype(np.uint64)
-    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    # finite float32 bit patterns are <= 0xFF7FFFFF, so the rounding add cannot wrap
+    rounded = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
     return rounded.astype(np.uint16)
 
 

@@ -1,0 +1,180 @@
+/*
+ * rfq.h -- C ABI of the B200 (sm_100a) Residual Fallback Quantization library.
+ *
+ * The operation (from "Activation Outliers Matter: Robust Recovery for Quantized
+ * Multimodal LLMs", abstract and section 1, the RFQ contribution paragraph):
+ * a linear layer's activation X is quantized to FP4, the full quantization error
+ * R = X - DQ(Q(X)) is quantized again by a second low-bit path, and the GEMM
+ * accumulates both contributions:
+ *
+ *     Y = (DQ(Q(X)) + DQ(Q(R))) . DQ(Q(W))^T
+ *
+ * with no threshold, nothing dropped and no architectural change to the layer.
+ * The FP4 format is MXFP4 (OCP Microscaling v1.0; the pages name it but stop
+ * before defining it, at section 3.1):
+ *   - blocks of 32 consecutive elements along K share one E8M0 scale byte
+ *     s = clamp(floor(log2(amax)) - 2, -127, 127) + 127 (0 for an all-zero block,
+ *     0xFF when the block holds a NaN or infinity);
+ *   - each element is an E2M1 code: bit 3 sign (copied from the input, so -0
+ *     encodes as 0x8), bits 2..0 the magnitude |x| * 2^-(s-127) rounded to the
+ *     nearest of {0, .5, 1, 1.5, 2, 3, 4, 6}, ties to even mantissa, values >= 6
+ *     saturating to 6;
+ *   - R is formed in fp32, where it is exact, and quantized by the same rule.
+ *
+ * Data layouts (all row-major, K contiguous, caller-owned device memory):
+ *   bf16 inputs   X [M][K], W [N][K]                      (2 bytes per element)
+ *   codes         [rows][K/2] bytes; element 2j in bits 3..0, 2j+1 in bits 7..4
+ *   scales        the layout the Blackwell block-scaled MMA reads: the plain
+ *                 [rows][K/32] scale matrix padded to rows_pad = ceil(rows/128)*128
+ *                 and kb_pad = ceil(K/32/4)*4 (padding bytes 0), cut into 512-byte
+ *                 atoms of 128 rows x 4 blocks stored with the block-tile index
+ *                 fastest; inside an atom (r, c) is at (r%32)*16 + (r/32)*4 + c.
+ *                 Size: rfq_scales_bytes(rows, K).
+ *   Y [M][N]      fp32 or bf16 (rfq_out_t), fully overwritten.
+ *
+ * Conventions for every call:
+ *   - Pointers are device pointers (cudaMalloc'd or equivalent) owned by the
+ *     caller; the library allocates no device memory and keeps no pointer after
+ *     returning.  Outputs must not alias inputs.
+ *   - Work is enqueued asynchronously on `stream` (0 = legacy default stream) on
+ *     the current device, which must be compute capability 10.0 (B200/B100).
+ *   - Arguments are checked before anything is launched; a failed check returns
+ *     a status and launches nothing.  RFQ_ERR_CUDA reports a launch error from
+ *     the CUDA runtime.  Faults inside a kernel surface at the caller's next
+ *     synchronization.  Spin-waits inside the GEMM are bounded; a wait that runs
+ *     out sets a device error word that rfq_check_device_error() reports.
+ *   - No C++ exception crosses this boundary.  All functions are thread-safe
+ *     (no global mutable host state besides a per-process cache of the device's
+ *     properties).
+ */
+#ifndef RFQ_H_
+#define RFQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as the CUDA runtime's stream handle; NULL means the default stream. */
+typedef struct CUstream_st* cudaStream_t;
+
+typedef enum {
+  RFQ_OK = 0,
+  RFQ_ERR_INVALID_ARG = 1,       /* NULL pointer, negative size, inconsistent pair */
+  RFQ_ERR_UNSUPPORTED_SHAPE = 2, /* K not a multiple of 32, N not a multiple of 8, too large */
+  RFQ_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
+  RFQ_ERR_UNSUPPORTED_DEVICE = 4,/* current device is not compute capability 10.0 */
+  RFQ_ERR_CUDA = 5,              /* CUDA runtime error at launch */
+  RFQ_ERR_TIMEOUT = 6,           /* a bounded device-side wait ran out (from rfq_check_device_error) */
+  RFQ_ERR_WORKSPACE = 7          /* workspace NULL or smaller than rfq_linear_workspace_bytes() */
+} rfq_status_t;
+
+typedef enum { RFQ_OUT_F32 = 0, RFQ_OUT_BF16 = 1 } rfq_out_t;
+
+/* Human-readable name of a status (static string, never NULL). */
+const char* rfq_status_string(rfq_status_t status);
+
+/* Bytes of a packed code array for a [rows][K] matrix: rows * K / 2.
+ * Returns 0 for negative sizes or K not a multiple of 32. */
+size_t rfq_codes_bytes(int64_t rows, int64_t K);
+
+/* Bytes of a scale array in the MMA layout: ceil(rows/128)*128 * ceil(K/128)*4.
+ * Returns 0 for negative sizes or K not a multiple of 32. */
+size_t rfq_scales_bytes(int64_t rows, int64_t K);
+
+/*
+ * rfq_quantize_mxfp4 -- the fused single-pass RFQ activation quantizer.
+ * Reads X once and writes Q(X) and, when the residual pointers are given, Q(R)
+ * with R = X - DQ(Q(X)) (the paper's "full quantization error" requantized by
+ * "a second low-bit quantization path", section 1).
+ *
+ *   x_bf16              [M][K] bf16, 16-byte aligned
+ *   qx_codes, qx_scales Q(X): rfq_codes_bytes(M, K) and rfq_scales_bytes(M, K) bytes
+ *   qr_codes, qr_scales Q(R): same sizes; both NULL = residual path off (plain
+ *                       MXFP4); exactly one NULL is RFQ_ERR_INVALID_ARG
+ * K must be a multiple of 32; M >= 0 (M == 0 or K == 0 launches nothing).
+ * Every byte of the scale arrays, padding included, is written.
+ */
+rfq_status_t rfq_quantize_mxfp4(const void* x_bf16, int64_t M, int64_t K,
+                                void* qx_codes, void* qx_scales,
+                                void* qr_codes, void* qr_scales,
+                                cudaStream_t stream);
+
+/*
+ * rfq_quantize_weight -- plain MXFP4 quantization of W [N][K] (no residual path:
+ * weight quantization is the secondary error source, section 1).  Same layouts
+ * and rules as rfq_quantize_mxfp4 with rows = N.  Done once per weight.
+ */
+rfq_status_t rfq_quantize_weight(const void* w_bf16, int64_t N, int64_t K,
+                                 void* qw_codes, void* qw_scales,
+                                 cudaStream_t stream);
+
+/*
+ * rfq_gemm -- the RFQ GEMM: Y = DQ(QX).DQ(QW)^T + DQ(QR).DQ(QW)^T, both terms
+ * accumulated in fp32 into one accumulator (equivalently one GEMM over the
+ * concatenated K, [QX | QR] against [QW | QW]); "requantize the activation
+ * residual during GEMM and accumulate its contribution" (section 1).
+ * qr_codes == qr_scales == NULL gives the plain MXFP4 GEMM (residual path off).
+ *
+ *   qx_*, qr_*   [M][K] operands as written by rfq_quantize_mxfp4
+ *   qw_*         [N][K] operand as written by rfq_quantize_weight
+ *   y            [M][N], y_type fp32 or bf16 (round to nearest even), 16-byte aligned
+ * K multiple of 32; N multiple of 8.  M == 0 or N == 0 launches nothing;
+ * K == 0 writes zeros.  Tensor cores: tcgen05 kind::mxf4 block-scaled MMAs.
+ */
+rfq_status_t rfq_gemm(const void* qx_codes, const void* qx_scales,
+                      const void* qr_codes, const void* qr_scales,
+                      const void* qw_codes, const void* qw_scales,
+                      int64_t M, int64_t N, int64_t K,
+                      void* y, rfq_out_t y_type, cudaStream_t stream);
+
+/* Workspace bytes rfq_linear needs for an [M][K] activation: codes and scales
+ * of Q(X) and, when use_residual, of Q(R), each sub-buffer 256-byte aligned. */
+size_t rfq_linear_workspace_bytes(int64_t M, int64_t K, int use_residual);
+
+/*
+ * rfq_linear -- the RFQ linear layer: rfq_quantize_mxfp4 of X into the caller's
+ * workspace, then rfq_gemm against the pre-quantized weight, on one stream
+ * ("requires no architectural modifications": a drop-in for the layer's GEMM).
+ *
+ *   x_bf16          [M][K] bf16
+ *   qw_codes/scales the weight as written by rfq_quantize_weight for [N][K]
+ *   y               [M][N] in y_type
+ *   use_residual    1 = RFQ (both terms), 0 = plain MXFP4
+ *   workspace       device buffer of at least rfq_linear_workspace_bytes(M, K,
+ *                   use_residual) bytes, 256-byte aligned; its contents on
+ *                   return are the quantized activation (unspecified layout)
+ */
+rfq_status_t rfq_linear(const void* x_bf16, int64_t M, int64_t K,
+                        const void* qw_codes, const void* qw_scales, int64_t N,
+                        void* y, rfq_out_t y_type, int use_residual,
+                        void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+
+/*
+ * rfq_check_device_error -- synchronize `stream`, then read and clear the current
+ * device's error word that bounded waits inside the kernels set.  Returns
+ * RFQ_OK, RFQ_ERR_TIMEOUT (a wait ran out; the kernel wrote no complete result),
+ * or RFQ_ERR_CUDA (the synchronization itself failed).  When detail is non-NULL
+ * it receives the raw word (0 = none; otherwise a code naming the wait).
+ */
+rfq_status_t rfq_check_device_error(cudaStream_t stream, int* detail);
+
+/*
+ * Testing hook for the bounded waits (no counterpart in the paper): the next
+ * rfq_gemm launched by this process makes the producer of its first CTA skip
+ * stage fill number `fill_index` (counted from 0 over that CTA's k-tiles), so
+ * the MMA warp's wait for that stage runs out after about 1.5 s; the kernel then
+ * drains its own copies and MMAs, frees its TMEM and returns, and
+ * rfq_check_device_error() reports RFQ_ERR_TIMEOUT.  fill_index < 0 clears a
+ * pending request.  Always returns RFQ_OK.
+ */
+rfq_status_t rfq_debug_skip_next_fill(int fill_index);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RFQ_H_ */

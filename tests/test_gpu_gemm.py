@@ -1,0 +1,145 @@
+"""Kernel 2 (RFQ block-scaled GEMM on tcgen05) and rfq_linear against the CPU oracle.
+
+Y_gpu must satisfy max|Y_gpu - Y_ref| <= 1e-5 * S (fp32 output), plus one bf16
+ulp for bf16 output, where Y_ref and S come from the oracle's own quantization
+of the same seeded bf16 inputs (nothing the GPU computed is fed to the oracle).
+"""
+import numpy as np
+import pytest
+
+from block_scaled_gemm_rfq_b200 import workloads as wl
+from helpers import assert_y_close, dev_bf16, y_to_numpy
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gemm(rfq, x_bits, w_bits, residual, out_dtype):
+    import torch
+    x, w = dev_bf16(x_bits), dev_bf16(w_bits)
+    qa = rfq.quantize_mxfp4_alloc(x, residual=residual)
+    qw = rfq.quantize_weight_alloc(w)
+    y = rfq.gemm_alloc(qa, qw, out_dtype=out_dtype, use_residual=residual)
+    torch.cuda.synchronize()
+    rfq.check_device_error()
+    return y_to_numpy(y)
+
+
+def run_linear(rfq, x_bits, w_bits, residual, out_dtype):
+    import torch
+    x, w = dev_bf16(x_bits), dev_bf16(w_bits)
+    qw = rfq.quantize_weight_alloc(w)
+    y = rfq.linear_alloc(x, qw, out_dtype=out_dtype, use_residual=residual)
+    torch.cuda.synchronize()
+    rfq.check_device_error()
+    return y_to_numpy(y)
+
+
+def test_tiny_rfq_linear_fp32(rfq, oracle):
+    import torch
+    w = wl.tiny(0)
+    Y, S, _ = oracle.rfq_linear(w.x_bits, w.w_bits, residual=True)
+    for runner in (run_gemm, run_linear):
+        y = runner(rfq, w.x_bits, w.w_bits, True, torch.float32)
+        assert_y_close(y, Y, S, bf16_out=False)
+
+
+def test_tiny_rfq_off(rfq, oracle):
+    import torch
+    w = wl.tiny(0)
+    Y, S, _ = oracle.rfq_linear(w.x_bits, w.w_bits, residual=False)
+    y = run_gemm(rfq, w.x_bits, w.w_bits, False, torch.float32)
+    assert_y_close(y, Y, S, bf16_out=False)
+
+
+def test_tiny_bf16_output(rfq, oracle):
+    import torch
+    w = wl.tiny(1)
+    Y, S, _ = oracle.rfq_linear(w.x_bits, w.w_bits, residual=True)
+    y = run_linear(rfq, w.x_bits, w.w_bits, True, torch.bfloat16)
+    assert_y_close(y, Y, S, bf16_out=True)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 64), (16, 16, 64), (127, 136, 96), (129, 264, 160), (300, 520, 1024),
+                                   (256, 256, 4096), (64, 512, 32), (200, 1000, 2080)])
+@pytest.mark.parametrize("residual", [True, False])
+def test_edge_shapes(rfq, oracle, M, N, K, residual):
+    import torch
+    x = wl.random_matrix(M, K, seed=M + 3 * N + 7 * K, scale=2.0)
+    w = wl.random_matrix(N, K, seed=M * N + K, scale=0.05)
+    Y, S, _ = oracle.rfq_linear(x, w, residual=residual)
+    y = run_gemm(rfq, x, w, residual, torch.float32)
+    assert_y_close(y, Y, S, bf16_out=False, what=f"Y[{M}x{N}x{K}]")
+
+
+def test_outlier_heavy_inputs(rfq, oracle):
+    """Large dynamic range inside a row: outlier channels x1000 and tiny channels."""
+    import torch
+    rng = np.random.default_rng(4)
+    X = rng.standard_t(3.0, (192, 512))
+    X[:, rng.choice(512, 10, replace=False)] *= 1000.0
+    X[:, rng.choice(512, 10, replace=False)] *= 1e-6
+    W = rng.normal(0, 0.02, (264, 512))
+    xb, wb = wl.f64_to_bf16_bits(X), wl.f64_to_bf16_bits(W)
+    Y, S, _ = oracle.rfq_linear(xb, wb, residual=True)
+    y = run_gemm(rfq, xb, wb, True, torch.float32)
+    assert_y_close(y, Y, S, bf16_out=False)
+
+
+def test_k_zero_writes_zeros(rfq):
+    import torch
+    y = torch.full((16, 16), 7.0, device="cuda")
+    empty = torch.empty(16, dtype=torch.uint8, device="cuda")
+    rfq.gemm(empty, empty, None, None, empty, empty, 16, 16, 0, y)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(y).item() == 0
+
+
+def _sampled_rows_check(rfq, oracle, wk, rows, residual=True):
+    """Full-size GEMM on the GPU; the oracle recomputes the sampled rows of Y (all
+    N columns) from its own quantization of those rows of X and of all of W.
+    S is taken over the sampled rows, which is <= the full-matrix S (stricter)."""
+    import torch
+    x_sub = wk.x_bits[rows]
+    qa = oracle.quantize_bf16(x_sub, residual=residual)
+    qw = oracle.quantize_bf16(wk.w_bits, residual=False)
+    A, B = oracle.rfq_operands(qa, qw, residual)
+    Y, absY = oracle.gemm_blas(A, B)
+    S = float(absY.max())
+    for out in (torch.float32, torch.bfloat16):
+        y = run_gemm(rfq, wk.x_bits, wk.w_bits, residual, out)
+        assert_y_close(y[rows], Y, S, bf16_out=(out == torch.bfloat16), what=f"{wk.name} {out}")
+
+
+def _sample(M, n, seed):
+    rng = np.random.default_rng(seed)
+    r = set(rng.choice(M, n, replace=False).tolist()) | {0, M - 1, 127, 128}
+    return np.array(sorted(i for i in r if i < M))
+
+
+def test_ffn_up_workload_sampled(rfq, oracle):
+    wk = wl.ffn_up(0)
+    _sampled_rows_check(rfq, oracle, wk, _sample(wk.M, 60, 1))
+
+
+def test_dit_ffn_workload_sampled(rfq, oracle):
+    wk = wl.dit_ffn(0)
+    _sampled_rows_check(rfq, oracle, wk, _sample(wk.M, 24, 2), residual=True)
+
+
+def test_dit_ffn_workload_rfq_off_sampled(rfq, oracle):
+    wk = wl.dit_ffn(0)
+    _sampled_rows_check(rfq, oracle, wk, _sample(wk.M, 24, 3), residual=False)
+
+
+@pytest.mark.parametrize("M", wl.SWEEP_M)
+def test_m_sweep_linear_sampled(rfq, oracle, M):
+    import torch
+    wk = wl.m_sweep(M)
+    rows = _sample(M, min(M, 32), M)
+    for residual in (True, False):
+        qa = oracle.quantize_bf16(wk.x_bits[rows], residual=residual)
+        qw = oracle.quantize_bf16(wk.w_bits, residual=False)
+        A, B = oracle.rfq_operands(qa, qw, residual)
+        Y, absY = oracle.gemm_blas(A, B)
+        y = run_linear(rfq, wk.x_bits, wk.w_bits, residual, torch.bfloat16)
+        assert_y_close(y[rows], Y, float(absY.max()), bf16_out=True, what=f"sweep M={M} res={residual}")
