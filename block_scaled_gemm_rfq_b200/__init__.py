@@ -18,7 +18,8 @@ import threading
 
 __all__ = [
     "RFQError", "load_library", "library_path", "codes_bytes", "scales_bytes", "linear_workspace_bytes",
-    "quantize_mxfp4", "quantize_weight", "gemm", "linear", "check_device_error", "debug_skip_next_fill",
+    "quantize_mxfp4", "quantize_weight", "gemm", "linear", "linear_static_workspace", "check_device_error",
+    "debug_skip_next_fill", "STATIC_WORKSPACE_BYTES",
     "QuantizedTensor", "quantize_mxfp4_alloc", "quantize_weight_alloc", "gemm_alloc", "linear_alloc",
     "EXPORTED_SYMBOLS", "OUT_F32", "OUT_BF16",
 ]
@@ -38,7 +39,11 @@ STATUS = {0: "RFQ_OK", 1: "RFQ_ERR_INVALID_ARG", 2: "RFQ_ERR_UNSUPPORTED_SHAPE",
 EXPORTED_SYMBOLS = (
     "rfq_status_string", "rfq_codes_bytes", "rfq_scales_bytes", "rfq_quantize_mxfp4", "rfq_quantize_weight",
     "rfq_gemm", "rfq_linear_workspace_bytes", "rfq_linear", "rfq_check_device_error", "rfq_debug_skip_next_fill",
+    "rfq_linear_static_workspace",
 )
+
+# Size of the library's fixed scratch array (RFQ_STATIC_WORKSPACE_BYTES in include/rfq.h).
+STATIC_WORKSPACE_BYTES = 32 << 20
 
 
 class RFQError(RuntimeError):
@@ -72,6 +77,7 @@ def load_library():
                 "rfq_linear": (I, [P, I64, I64, P, P, I64, P, I, I, P, SZ, P]),
                 "rfq_check_device_error": (I, [P, ctypes.POINTER(ctypes.c_int)]),
                 "rfq_debug_skip_next_fill": (I, [I]),
+                "rfq_linear_static_workspace": (I, [P, I64, I64, P, P, I64, P, I, I, P]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(lib, name)
@@ -140,6 +146,18 @@ def linear(x, qw_codes, qw_scales, N, y, workspace, use_residual=True, stream=No
     _check(load_library().rfq_linear(_ptr(x), M, K, _ptr(qw_codes), _ptr(qw_scales), N, _ptr(y), y_type,
                                      int(bool(use_residual)), _ptr(workspace), workspace.numel(), _stream(stream)),
            "rfq_linear")
+
+
+def linear_static_workspace(x, qw_codes, qw_scales, N, y, use_residual=True, stream=None):
+    """rfq_linear_static_workspace: the RFQ linear layer for callers that cannot allocate
+    device memory; the quantized activation goes into the library's fixed 32 MiB scratch
+    array (see include/rfq.h for the size limit and the no-overlap rule)."""
+    import torch
+    M, K = x.shape
+    y_type = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
+    _check(load_library().rfq_linear_static_workspace(_ptr(x), M, K, _ptr(qw_codes), _ptr(qw_scales), N, _ptr(y),
+                                                      y_type, int(bool(use_residual)), _stream(stream)),
+           "rfq_linear_static_workspace")
 
 
 def check_device_error(stream=None):

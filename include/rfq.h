@@ -154,6 +154,42 @@ rfq_status_t rfq_linear(const void* x_bf16, int64_t M, int64_t K,
                         cudaStream_t stream);
 
 /*
+ * Size of the fixed scratch array used by rfq_linear_static_workspace: 32 MiB of
+ * device memory, reserved on every GPU that loads this library and kept until
+ * the process exits.
+ */
+#define RFQ_STATIC_WORKSPACE_BYTES (32u << 20)
+
+/*
+ * rfq_linear_static_workspace -- rfq_linear without a caller-provided workspace
+ * (the paper has no counterpart; this is a deployment convenience).
+ *
+ * For callers that cannot allocate device memory when they run the layer, e.g. a
+ * plug-in inside a host application that owns the device's memory pool and
+ * forbids raw cudaMalloc, or a latency-critical loop where allocating (which can
+ * synchronize the device) is not allowed.  The quantized activation goes into a
+ * fixed scratch array inside this library's own device memory instead; this
+ * call allocates nothing.  Arguments, layouts and results are those of
+ * rfq_linear; the caller still provides X, the quantized weight and Y.
+ *
+ *   - Size limit: rfq_linear_workspace_bytes(M, K, use_residual) must not exceed
+ *     RFQ_STATIC_WORKSPACE_BYTES (about M*K <= 31.5 Mi elements with the residual
+ *     path, 63 Mi without); larger problems return RFQ_ERR_UNSUPPORTED_SHAPE and
+ *     launch nothing.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (once; cached afterwards).  Make that first call before any stream
+ *     capture on the device.
+ *   - Every call on a device shares the one array and it keeps the last call's
+ *     contents.  Calls whose GPU work can overlap (different streams without
+ *     ordering between them, or several host threads) race on it and corrupt
+ *     each other's results; serialize them, e.g. on one stream.
+ */
+rfq_status_t rfq_linear_static_workspace(const void* x_bf16, int64_t M, int64_t K,
+                                         const void* qw_codes, const void* qw_scales, int64_t N,
+                                         void* y, rfq_out_t y_type, int use_residual,
+                                         cudaStream_t stream);
+
+/*
  * rfq_check_device_error -- synchronize `stream`, then read and clear the current
  * device's error word that bounded waits inside the kernels set.  Returns
  * RFQ_OK, RFQ_ERR_TIMEOUT (a wait ran out; the kernel wrote no complete result),
