@@ -440,6 +440,35 @@ def run_reference(args):
     }
 
 
+def run_single_kernel(args):
+    """--kernel quantize|gemm|linear: time one kernel on a chosen shape (for sweeps and
+    profiles); prints one JSON line with per-launch times."""
+    import numpy as np
+    import torch
+
+    import block_scaled_gemm_rfq_b200 as rfq
+    from block_scaled_gemm_rfq_b200 import workloads as wl
+    rfq.load_library()
+    M, K, N = args.M, args.K, args.N
+    x = to_device_bf16(wl.random_matrix(M, K, seed=1, scale=2.0))
+    w = to_device_bf16(wl.random_matrix(N, K, seed=2, scale=0.05)) if args.kernel != "quantize" else x[:8]
+    step = RfqStep(rfq, x, w, residual=not args.no_rfq)
+    step.quantize_w()
+    step.quantize_x()
+    fn = {"quantize": step.quantize_x, "gemm": step.gemm, "linear": step.run}[args.kernel]
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    t = time_kernel(fn, args.steps, lambda: flush_buf.zero_())
+    rfq.check_device_error()
+    ms = statistics.mean(t)
+    out = {"kernel": args.kernel, "M": M, "K": K, "N": N, "rfq": not args.no_rfq, "iters": args.steps,
+           "ms_mean": ms, "ms_min": min(t)}
+    if args.kernel == "quantize":
+        out["gbs"] = quantize_bytes(M, K, not args.no_rfq) / (ms * 1e-3) / 1e9
+    else:
+        out["tflops_executed"] = (2.0 if args.no_rfq else 4.0) * M * N * K / (ms * 1e-3) / 1e12
+    print(json.dumps(out))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -449,9 +478,19 @@ def main():
     ap.add_argument("--all-configs", action="store_true", help="also time the DiT FFN GEMM and the M sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--kernel", choices=["quantize", "gemm", "linear"], default=None,
+                    help="time one kernel on --M/--N/--K instead of the benchmark step")
+    ap.add_argument("--M", type=int, default=4096)
+    ap.add_argument("--N", type=int, default=12288)
+    ap.add_argument("--K", type=int, default=4096)
+    ap.add_argument("--no-rfq", action="store_true", help="with --kernel: residual path off")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+
+    if args.kernel:
+        run_single_kernel(args)
+        return
 
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:

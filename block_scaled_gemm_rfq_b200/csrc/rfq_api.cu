@@ -65,8 +65,12 @@ rfq_status_t current_device(int* num_sms) {
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// Limits: rows and K fit the kernels' 32-bit tile coordinates, and a matrix holds
+// at most 2^31 - 64 blocks of 32 elements (the quantizer's TMA row coordinate,
+// which runs up to 31 blocks past the last one).
 bool shape_ok(int64_t rows, int64_t K) {
-  return rows >= 0 && K >= 0 && (K % 32) == 0 && rows <= (int64_t(1) << 31) - 1 && K <= (int64_t(1) << 31) - 32;
+  return rows >= 0 && K >= 0 && (K % 32) == 0 && rows <= (int64_t(1) << 31) - 1 && K <= (int64_t(1) << 31) - 32 &&
+         (K == 0 || rows <= ((int64_t(1) << 31) - 64) / (K / 32));
 }
 
 rfq_status_t check_quantize_args(const void* x, int64_t M, int64_t K, const void* qc, const void* qs, const void* rc,
@@ -92,7 +96,7 @@ rfq_status_t quantize_impl(const void* x, int64_t M, int64_t K, void* qc, void* 
     // No blocks: the scale arrays have no bytes (rfq_scales_bytes == 0); nothing to do.
     return RFQ_OK;
   }
-  return from_cuda(rfq::launch_quantize(x, M, K, qc, qs, rc, rs, sms, stream));
+  return from_cuda(rfq::launch_quantize(x, M, K, qc, qs, rc, rs, sms, g_encode_tiled, stream));
 }
 
 rfq_status_t gemm_impl(const void* qxc, const void* qxs, const void* qrc, const void* qrs, const void* qwc,
@@ -197,8 +201,10 @@ rfq_status_t rfq_linear(const void* x_bf16, int64_t M, int64_t K, const void* qw
 rfq_status_t rfq_check_device_error(cudaStream_t stream, int* detail) {
   if (detail) *detail = 0;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return RFQ_ERR_CUDA;
-  unsigned int v = 0;
+  unsigned int v = 0, q = 0;
   if (rfq::read_and_clear_device_error(&v) != cudaSuccess) return RFQ_ERR_CUDA;
+  if (rfq::read_and_clear_quant_error(&q) != cudaSuccess) return RFQ_ERR_CUDA;
+  if (v == 0) v = q;
   if (detail) *detail = static_cast<int>(v);
   return v ? RFQ_ERR_TIMEOUT : RFQ_OK;
 }

@@ -20,8 +20,9 @@
 //               (tcgen05.cp 32x128b.warpx4) and issues 2 + 2 MMAs of K = 64;
 //               tcgen05.commit frees the stage and, at the end of a tile,
 //               signals the epilogue;
-//   warps 2..5  epilogue: TMEM -> registers (tcgen05.ld 32x32b) -> fp32/bf16 ->
-//               global, one accumulator row per thread.
+//   warps 2..9  epilogue: TMEM -> registers (tcgen05.ld 32x32b, 128 columns per
+//               warp), release of the accumulator, then fp32/bf16 -> global,
+//               one accumulator row per thread, overlapping the next mainloop.
 // Every mbarrier wait is bounded (rfq_ptx.cuh); a wait that runs out records an
 // error code, raises the CTA's abort flag and the CTA tears down cleanly (its
 // copies and MMAs drained, its TMEM freed).  No TMA multicast is used.
@@ -45,7 +46,7 @@ constexpr int kBN = 256;               // rows of W / columns of Y per tile (MMA
 constexpr int kBK = 128;               // K elements per stage
 constexpr int kBKBytes = kBK / 2;      // packed FP4: 64 bytes per row per stage
 constexpr int kStages = 6;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;        // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;        // 256 fp32 columns: the 128 x 256 accumulator
 constexpr uint32_t kSfaXCol = 256;     // 4 columns: scales of QX for 128 rows x 4 blocks
@@ -135,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);
+    mbar_init(acc_empty, 8);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -259,52 +260,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    const int quad = warp & 3;  // TMEM lanes this warp may access: 32*quad .. 32*quad+31
+    // 8 warps: two per TMEM lane quadrant, each owning 128 of the 256 columns.
+    // The accumulator is copied to registers first and released to the MMA warp
+    // at once, so converting and storing Y overlaps the next tile's mainloop.
+    const int quad = warp & 3;                // TMEM lanes this warp may access: 32*quad .. 32*quad+31
+    const int half = (warp - 2) >> 2;         // columns [128*half, 128*half + 128)
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       const int mb = tile / p.num_nb;
       const int nb = tile - mb * p.num_nb;
       if (!mbar_wait(acc_full, acc_phase, abort_flag, &g_device_error, kErrWaitAccFull)) break;
       tc_fence_after();
-      const int row = mb * kBM + quad * 32 + lane;
-      const bool row_ok = row < p.M;
-#pragma unroll 1
-      for (int c0 = 0; c0 < kBN; c0 += 32) {
-        uint32_t v[32];
-        tmem_load_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + kAccCol + c0, v);
-        tmem_wait_ld();
-        const int col = nb * kBN + c0;
-        if (row_ok) {
-          if (kBf16Out) {
-            __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(row) * p.N + col;
+      uint32_t v[4][32];
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + kAccCol + half * 128;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              if (col + 8 * i < p.N) {
-                uint4 pk;
-                uint32_t* pw = reinterpret_cast<uint32_t*>(&pk);
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                  __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 2 * h]),
-                                                            __uint_as_float(v[8 * i + 2 * h + 1]));
-                  pw[h] = *reinterpret_cast<uint32_t*>(&b2);
-                }
-                *reinterpret_cast<uint4*>(yrow + 8 * i) = pk;
-              }
-            }
-          } else {
-            float* yrow = static_cast<float*>(p.y) + static_cast<int64_t>(row) * p.N + col;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              if (col + 4 * i < p.N)
-                *reinterpret_cast<uint4*>(yrow + 4 * i) = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            }
-          }
-        }
-      }
+      for (int c = 0; c < 4; ++c) tmem_load_32x32b_x32(taddr + 32 * c, v[c]);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
       acc_phase ^= 1u;
+
+      const int row = mb * kBM + quad * 32 + lane;
+      const int col0 = nb * kBN + half * 128;
+      if (row < p.M) {
+        if (kBf16Out) {
+          __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(row) * p.N + col0;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (col0 + 8 * i < p.N) {
+              uint32_t pw[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const int e = 8 * i + 2 * h;
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[e >> 5][e & 31]),
+                                                          __uint_as_float(v[(e + 1) >> 5][(e + 1) & 31]));
+                pw[h] = *reinterpret_cast<uint32_t*>(&b2);
+              }
+              *reinterpret_cast<uint4*>(yrow + 8 * i) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+            }
+          }
+        } else {
+          float* yrow = static_cast<float*>(p.y) + static_cast<int64_t>(row) * p.N + col0;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int e = 4 * i;
+            if (col0 + e < p.N)
+              *reinterpret_cast<uint4*>(yrow + e) =
+                  make_uint4(v[e >> 5][e & 31], v[e >> 5][(e & 31) + 1], v[e >> 5][(e & 31) + 2], v[e >> 5][(e & 31) + 3]);
+          }
+        }
+      }
     }
   }
 

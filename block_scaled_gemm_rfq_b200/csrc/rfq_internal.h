@@ -9,8 +9,9 @@
 namespace rfq {
 
 // Kernel 1: fused quantizer.  qr_codes == nullptr selects plain MXFP4.
+// `encode_tiled` is the driver's cuTensorMapEncodeTiled.
 cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, void* qx_codes, void* qx_scales, void* qr_codes,
-                            void* qr_scales, int num_sms, cudaStream_t stream);
+                            void* qr_scales, int num_sms, void* encode_tiled, cudaStream_t stream);
 
 // Kernel 2: RFQ GEMM.  qr_codes == nullptr selects the plain MXFP4 GEMM.
 // `encode_tiled` is the driver's cuTensorMapEncodeTiled.  `skip_fill` >= 0 makes
@@ -20,7 +21,8 @@ cudaError_t launch_gemm(const void* qx_codes, const void* qx_scales, const void*
                         const void* qw_codes, const void* qw_scales, int64_t M, int64_t N, int64_t K, void* y,
                         bool y_bf16, int num_sms, void* encode_tiled, int skip_fill, cudaStream_t stream);
 
-// Read and clear the device error word of the current device.
+// Read and clear the device error words (GEMM and quantizer) of the current device.
 cudaError_t read_and_clear_device_error(unsigned int* value);
+cudaError_t read_and_clear_quant_error(unsigned int* value);
 
 }  // namespace rfq

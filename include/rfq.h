@@ -194,7 +194,9 @@ rfq_status_t rfq_linear_static_workspace(const void* x_bf16, int64_t M, int64_t 
  * device's error word that bounded waits inside the kernels set.  Returns
  * RFQ_OK, RFQ_ERR_TIMEOUT (a wait ran out; the kernel wrote no complete result),
  * or RFQ_ERR_CUDA (the synchronization itself failed).  When detail is non-NULL
- * it receives the raw word (0 = none; otherwise a code naming the wait).
+ * it receives the raw word (0 = none; 1..5 a wait inside rfq_gemm: 1 stage
+ * load, 2 free stage, 3 accumulator ready, 4 accumulator free, 5 teardown;
+ * 6 a wait of the quantizer for its TMA load).
  */
 rfq_status_t rfq_check_device_error(cudaStream_t stream, int* detail);
 
