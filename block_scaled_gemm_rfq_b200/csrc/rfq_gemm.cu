@@ -11,21 +11,28 @@
 // reusing the QW tile already in shared memory, so the residual doubles the work
 // on the tensor pipe (K -> 2K) and costs no extra pass over Y.
 //
-// Structure (one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 0      TMA producer: per k-tile (128 elements = 64 bytes per row) it
-//               loads the QX, QR and QW code tiles (2-D tensor maps, 64-byte
-//               swizzle) and their 512-byte scale atoms (1-D bulk copies) into a
-//               kStages-deep shared-memory ring guarded by mbarriers;
-//   warp 1      MMA issuer (one thread): copies the stage's scale atoms into TMEM
-//               (tcgen05.cp 32x128b.warpx4) and issues 2 + 2 MMAs of K = 64;
-//               tcgen05.commit frees the stage and, at the end of a tile,
-//               signals the epilogue;
-//   warps 2..9  epilogue: TMEM -> registers (tcgen05.ld 32x32b, 128 columns per
-//               warp), release of the accumulator, then fp32/bf16 -> global,
-//               one accumulator row per thread, overlapping the next mainloop.
+// Two variants of one persistent, warp-specialized kernel:
+//   kPair = 1  one CTA per 128 x 256 output tile (MMA M = 128, cta_group::1);
+//   kPair = 2  a cluster of two CTAs per 256 x 256 tile (MMA M = 256,
+//              cta_group::2): each CTA loads its own 128 rows of QX/QR and half
+//              of the QW tile, the leader CTA issues the MMAs for the pair and
+//              the tensor cores read the QW halves from both CTAs' shared
+//              memory, so each SM moves ~25 % fewer operand bytes per MMA.
+// Roles (per CTA):
+//   warp 0      TMA producer: per k-tile (256 elements = 128 bytes per row) the
+//               code tiles (2-D maps, 128-byte swizzle) and the stage's scale
+//               atoms (one 4-D box per operand) into a kStages-deep ring;
+//               out-of-range rows/atoms are zero-filled by the TMA unit;
+//   warp 1      MMA issuer (one thread of the leader CTA): copies the stage's
+//               scale atoms to TMEM (tcgen05.cp 32x128b.warpx4) and issues 4 + 4
+//               MMAs of K = 64; tcgen05.commit frees the stage and, at the end of
+//               a tile, signals the epilogues;
+//   warps 2..9  epilogue: TMEM -> registers (128 columns per warp), release of
+//               the accumulator, then fp32/bf16 -> global, one row per thread,
+//               overlapping the next tile's mainloop.
 // Every mbarrier wait is bounded (rfq_ptx.cuh); a wait that runs out records an
-// error code, raises the CTA's abort flag and the CTA tears down cleanly (its
-// copies and MMAs drained, its TMEM freed).  No TMA multicast is used.
+// error code, raises the CTA's abort flag and the CTA tears down cleanly.  No TMA
+// multicast is used anywhere (the pair's loads each fill their own CTA).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -41,57 +48,67 @@ __device__ unsigned int g_device_error = 0;
 
 namespace {
 
-constexpr int kBM = 128;               // rows of X / Y per tile (MMA M)
-constexpr int kBN = 256;               // rows of W / columns of Y per tile (MMA N)
-constexpr int kBK = 128;               // K elements per stage
-constexpr int kBKBytes = kBK / 2;      // packed FP4: 64 bytes per row per stage
-constexpr int kStages = 6;
-constexpr int kThreads = 320;        // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kBM = 128;               // rows of X / Y per CTA (MMA M per CTA)
+constexpr int kBN = 256;               // columns of Y per tile (MMA N)
+constexpr int kBK = 256;               // K elements per stage (2 scale atoms of 128)
+constexpr int kBKBytes = kBK / 2;      // packed FP4: 128 bytes per row per stage
+constexpr int kThreads = 320;          // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCol = 0;        // 256 fp32 columns: the 128 x 256 accumulator
-constexpr uint32_t kSfaXCol = 256;     // 4 columns: scales of QX for 128 rows x 4 blocks
-constexpr uint32_t kSfaRCol = 260;     // 4 columns: scales of QR
-constexpr uint32_t kSfbCol = 264;      // 8 columns: scales of QW for 256 rows x 4 blocks
+constexpr uint32_t kAccCol = 0;        // 256 fp32 columns: the 128 x 256 accumulator of this CTA
+// Scale factors in TMEM: one 32-column slot per pipeline stage (from column 256),
+// so a stage's tcgen05.cp never overwrites scales that queued MMAs still read.
+// A slot holds the stage's 2 scale atoms (k-atoms a = 0, 1; 128 K each) of:
+constexpr uint32_t kSfBase = 256;
+constexpr uint32_t kSfSlot = 32;
+constexpr uint32_t kSfaXCol = 0;       // +4a..4a+3:   QX, this CTA's 128 rows
+constexpr uint32_t kSfaRCol = 8;       // +8+4a..:     QR
+constexpr uint32_t kSfbCol = 16;       // +16+8a..+7:  QW, the tile's 256 rows (2 row atoms)
+constexpr uint32_t kSmemLimit = 232448;
 
-constexpr uint32_t kATileBytes = kBM * kBKBytes;   // 8 KiB
-constexpr uint32_t kBTileBytes = kBN * kBKBytes;   // 16 KiB
-constexpr uint32_t kOffA = 0;
-constexpr uint32_t kOffR = kOffA + kATileBytes;
-constexpr uint32_t kOffB = kOffR + kATileBytes;
-constexpr uint32_t kOffSfaX = kOffB + kBTileBytes;
-constexpr uint32_t kOffSfaR = kOffSfaX + 512;
-constexpr uint32_t kOffSfb = kOffSfaR + 512;
-constexpr uint32_t kStageBytes = kOffSfb + 1024;   // 34 KiB, a multiple of 1 KiB
-constexpr uint32_t kBarrierBytes = 256;
-constexpr uint32_t kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;  // + alignment slack
-
-static_assert(kStageBytes % 1024 == 0, "stage buffers must keep 1 KiB alignment");
-static_assert(kSmemBytes <= 232448, "exceeds the 227 KiB shared-memory limit");
+template <int kPair>
+struct Layout {
+  static constexpr uint32_t kATile = kBM * kBKBytes;                 // 16 KiB
+  static constexpr uint32_t kBTile = (kBN / kPair) * kBKBytes;       // 32 KiB (single) or 16 KiB (pair)
+  static constexpr uint32_t kOffA = 0;
+  static constexpr uint32_t kOffR = kOffA + kATile;
+  static constexpr uint32_t kOffB = kOffR + kATile;
+  static constexpr uint32_t kOffSfaX = kOffB + kBTile;               // 2 atoms (k-atom 0, 1)
+  static constexpr uint32_t kOffSfaR = kOffSfaX + 1024;
+  static constexpr uint32_t kOffSfb = kOffSfaR + 1024;               // [row atom lo, hi][k-atom 0, 1]
+  static constexpr uint32_t kStage = kOffSfb + 2048;
+  static constexpr uint32_t kBarrierBytes = 256;
+  static constexpr int kStages = static_cast<int>((kSmemLimit - 1024 - kBarrierBytes) / kStage);
+  static constexpr uint32_t kSmem = kStages * kStage + kBarrierBytes + 1024;
+  static_assert(kStage % 1024 == 0, "stage buffers must keep 1 KiB alignment");
+  static_assert(kSmem <= kSmemLimit, "exceeds the 227 KiB shared-memory limit");
+  static_assert((2 * kStages + 3) * 8 + 8 <= kBarrierBytes, "barrier area too small");
+  static_assert(kSfBase + kStages * kSfSlot <= kTmemCols, "scale slots exceed TMEM");
+};
 
 struct GemmParams {
-  const uint8_t* sfa_x;
-  const uint8_t* sfa_r;
-  const uint8_t* sfb;
   void* y;
   int M;
   int N;
-  int num_kt;            // k-tiles of 128 elements
-  int atoms_per_rowtile; // scale atoms per 128-row tile = ceil(K/128)
+  int num_kt;            // k-tiles of 256 elements
   int num_nb;            // tiles along N
-  int num_tiles;
-  int b_rowtiles;        // ceil(N/128): scale atoms of W along N
+  int num_tiles;         // tiles (kPair = 1) or pair tiles (kPair = 2)
   int skip_fill;         // fault injection (-1 = off)
 };
 
-// Shared-memory matrix descriptor (tcgen05): K-major operand, 64-byte swizzle,
-// rows of 64 bytes, 8-row groups 512 bytes apart.
+struct Maps {
+  CUtensorMap x, r, w;           // codes: [rows][K/2] bytes, box 128 B x (128 | 256 | 128) rows, 128-byte swizzle
+  CUtensorMap sx, sr, sw;        // scales: [row tiles][k atoms][2][256 B]; box = 2 k-atoms of 1 (A) or 2 (B) row tiles
+};
+
+// Shared-memory matrix descriptor (tcgen05): K-major operand, 128-byte swizzle,
+// rows of 128 bytes, 8-row groups 1024 bytes apart.
 __device__ __forceinline__ uint64_t operand_desc(const void* p) {
   const uint64_t addr = smem_addr(p);
   return ((addr >> 4) & 0x3FFFull)     // start address
          | (1ull << 16)                // leading byte offset (unused for swizzled K-major)
-         | ((512ull >> 4) << 32)       // stride byte offset: 8 rows x 64 B
+         | ((1024ull >> 4) << 32)      // stride byte offset: 8 rows x 128 B
          | (1ull << 46)                // descriptor version (sm_100)
-         | (4ull << 61);               // layout: 64-byte swizzle
+         | (2ull << 61);               // layout: 128-byte swizzle
 }
 
 // Descriptor of a 512-byte scale atom as 32 rows x 16 bytes, no swizzle, 8-row
@@ -102,26 +119,27 @@ __device__ __forceinline__ uint64_t scale_desc(const void* p) {
 }
 
 // Instruction descriptor of kind::mxf4 with E8M0 scales: E2M1 x E2M1, both
-// K-major, M = 128, N = 256, scale-factor byte selectors for A and B.
+// K-major, M = 128 * kPair, N = 256, scale-factor byte selectors for A and B.
+template <int kPair>
 __device__ __forceinline__ uint32_t mma_idesc(uint32_t sf_id) {
-  return (sf_id << 4)                  // B scale-factor id
-         | (1u << 7)                   // A format E2M1
-         | (1u << 10)                  // B format E2M1
-         | (uint32_t(kBN >> 3) << 17)  // N / 8
-         | (1u << 23)                  // scale type UE8M0
-         | (uint32_t(kBM >> 4) << 24)  // M / 16
-         | (sf_id << 29);              // A scale-factor id
+  return (sf_id << 4)                            // B scale-factor id
+         | (1u << 7)                             // A format E2M1
+         | (1u << 10)                            // B format E2M1
+         | (uint32_t(kBN >> 3) << 17)            // N / 8
+         | (1u << 23)                            // scale type UE8M0
+         | (uint32_t((kBM * kPair) >> 4) << 24)  // M / 16
+         | (sf_id << 29);                        // A scale-factor id
 }
 
-template <bool kResidual, bool kBf16Out>
+template <int kPair, bool kResidual, bool kBf16Out>
 __global__ void __launch_bounds__(kThreads, 1)
-    rfq_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_r,
-                    const __grid_constant__ CUtensorMap tm_w, const GemmParams p) {
+    rfq_gemm_kernel(const __grid_constant__ Maps maps, const GemmParams p) {
+  using L = Layout<kPair>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* acc_full = empty + kStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStage);
+  uint64_t* empty = full + L::kStages;
+  uint64_t* acc_full = empty + L::kStages;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -129,29 +147,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = kPair == 2 ? cluster_cta_rank() : 0u;     // 0 = leader of the pair
+  const bool leader = rank == 0;
+  const int unit = kPair == 2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int num_units = kPair == 2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 8);
+    mbar_init(acc_empty, 8 * kPair);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tm_x);
-    prefetch_tmap(&tm_w);
-    if (kResidual) prefetch_tmap(&tm_r);
+    prefetch_tmap(&maps.x);
+    prefetch_tmap(&maps.w);
+    prefetch_tmap(&maps.sx);
+    prefetch_tmap(&maps.sw);
+    if (kResidual) {
+      prefetch_tmap(&maps.r);
+      prefetch_tmap(&maps.sr);
+    }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_g<kPair>(tmem_slot, kTmemCols);
+    tmem_relinquish_g<kPair>();
   }
   tc_fence_before();
-  __syncthreads();
+  if (kPair == 2) cluster_sync();   // the peer's loads may signal our barriers from here on
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -161,53 +189,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0;
       uint32_t filled = 0, last_parity = 0;
       int fill = 0;
-      const uint32_t sfb_atoms_full = 2;
-      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      // Bytes one CTA loads per stage; the leader arms its full barrier with the
+      // bytes of both CTAs of a pair (the peer's copies complete on it too).
+      const uint32_t bytes_cta = L::kATile + L::kBTile + 1024u + 2048u + (kResidual ? L::kATile + 1024u : 0u);
+      const uint32_t bytes = bytes_cta * kPair;
+      for (int tile = unit; tile < p.num_tiles; tile += num_units) {
         const int mb = tile / p.num_nb;
         const int nb = tile - mb * p.num_nb;
-        const bool b_hi = (2 * nb + 1) < p.b_rowtiles;
-        const uint32_t bytes = kATileBytes + kBTileBytes + 512u + 512u * (b_hi ? sfb_atoms_full : 1u) +
-                               (kResidual ? kATileBytes + 512u : 0u);
-        const uint8_t* sfa_x_row = p.sfa_x + static_cast<int64_t>(mb) * p.atoms_per_rowtile * 512;
-        const uint8_t* sfa_r_row = kResidual ? p.sfa_r + static_cast<int64_t>(mb) * p.atoms_per_rowtile * 512 : nullptr;
-        const uint8_t* sfb_lo = p.sfb + static_cast<int64_t>(2 * nb) * p.atoms_per_rowtile * 512;
-        const uint8_t* sfb_hi = sfb_lo + static_cast<int64_t>(p.atoms_per_rowtile) * 512;
+        const int row_a = (mb * kPair + static_cast<int>(rank)) * kBM;       // this CTA's rows of X
+        const int row_b = nb * kBN + static_cast<int>(rank) * (kBN / kPair); // this CTA's rows of W
+        const int rt_a = mb * kPair + static_cast<int>(rank);                // this CTA's 128-row scale tile
         for (int kt = 0; kt < p.num_kt; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, &g_device_error, kErrWaitEmpty)) goto producer_done;
           if (!(fill == p.skip_fill && blockIdx.x == 0)) {
-            uint8_t* st = smem + stage * kStageBytes;
-            mbar_arrive_expect_tx(&full[stage], bytes);
-            tma_load_2d(st + kOffA, &tm_x, &full[stage], kt * kBKBytes, mb * kBM);
-            if (kResidual) tma_load_2d(st + kOffR, &tm_r, &full[stage], kt * kBKBytes, mb * kBM);
-            tma_load_2d(st + kOffB, &tm_w, &full[stage], kt * kBKBytes, nb * kBN);
-            bulk_load(st + kOffSfaX, sfa_x_row + kt * 512, 512, &full[stage]);
-            if (kResidual) bulk_load(st + kOffSfaR, sfa_r_row + kt * 512, 512, &full[stage]);
-            bulk_load(st + kOffSfb, sfb_lo + kt * 512, 512, &full[stage]);
-            if (b_hi) bulk_load(st + kOffSfb + 512, sfb_hi + kt * 512, 512, &full[stage]);
+            uint8_t* st = smem + stage * L::kStage;
+            if constexpr (kPair == 2) {
+              const uint32_t bar = map_to_cta(smem_addr(&full[stage]), 0);
+              if (leader) mbar_arrive_expect_tx(&full[stage], bytes);
+              tma_load_2d_pair(st + L::kOffA, &maps.x, bar, kt * kBKBytes, row_a);
+              if (kResidual) tma_load_2d_pair(st + L::kOffR, &maps.r, bar, kt * kBKBytes, row_a);
+              tma_load_2d_pair(st + L::kOffB, &maps.w, bar, kt * kBKBytes, row_b);
+              tma_load_4d_pair(st + L::kOffSfaX, &maps.sx, bar, 0, 0, 2 * kt, rt_a);
+              if (kResidual) tma_load_4d_pair(st + L::kOffSfaR, &maps.sr, bar, 0, 0, 2 * kt, rt_a);
+              tma_load_4d_pair(st + L::kOffSfb, &maps.sw, bar, 0, 0, 2 * kt, 2 * nb);
+            } else {
+              mbar_arrive_expect_tx(&full[stage], bytes);
+              tma_load_2d(st + L::kOffA, &maps.x, &full[stage], kt * kBKBytes, row_a);
+              if (kResidual) tma_load_2d(st + L::kOffR, &maps.r, &full[stage], kt * kBKBytes, row_a);
+              tma_load_2d(st + L::kOffB, &maps.w, &full[stage], kt * kBKBytes, row_b);
+              tma_load_4d(st + L::kOffSfaX, &maps.sx, &full[stage], 0, 0, 2 * kt, rt_a);
+              if (kResidual) tma_load_4d(st + L::kOffSfaR, &maps.sr, &full[stage], 0, 0, 2 * kt, rt_a);
+              tma_load_4d(st + L::kOffSfb, &maps.sw, &full[stage], 0, 0, 2 * kt, 2 * nb);
+            }
             filled |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           }
           ++fill;
-          if (++stage == kStages) {
+          if (++stage == static_cast<uint32_t>(L::kStages)) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
     producer_done:
-      // Teardown: every copy this thread issued must have landed before exit.
-      for (int s = 0; s < kStages; ++s)
-        if (filled & (1u << s)) {
-          int never = 0;
-          mbar_wait(&full[s], (last_parity >> s) & 1u, &never, &g_device_error, kErrWaitDrain);
-        }
+      // Teardown: every copy armed on this CTA's barriers must have landed (for a
+      // pair the leader's barriers also count the peer's copies).
+      if (leader)
+        for (int s = 0; s < L::kStages; ++s)
+          if (filled & (1u << s)) {
+            int never = 0;
+            mbar_wait(&full[s], (last_parity >> s) & 1u, &never, &g_device_error, kErrWaitDrain);
+          }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ------------------------------------------------------------ MMA issuer
       uint32_t stage = 0, phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+      for (int tile = unit; tile < p.num_tiles && ok; tile += num_units) {
         if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag, &g_device_error, kErrWaitAccEmpty)) {
           ok = false;
           break;
@@ -219,41 +258,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint8_t* st = smem + stage * kStageBytes;
-          tmem_copy_32x128b_warpx4(tmem + kSfaXCol, scale_desc(st + kOffSfaX));
-          if (kResidual) tmem_copy_32x128b_warpx4(tmem + kSfaRCol, scale_desc(st + kOffSfaR));
-          tmem_copy_32x128b_warpx4(tmem + kSfbCol, scale_desc(st + kOffSfb));
-          tmem_copy_32x128b_warpx4(tmem + kSfbCol + 4, scale_desc(st + kOffSfb + 512));
-          const uint64_t da = operand_desc(st + kOffA);
-          const uint64_t db = operand_desc(st + kOffB);
+          const uint8_t* st = smem + stage * L::kStage;
+          const uint32_t sf = tmem + kSfBase + stage * kSfSlot;
 #pragma unroll
-          for (uint32_t j = 0; j < 2; ++j) {
-            const uint32_t sf = 2u * j;  // MMA j uses scale bytes 2j, 2j+1 of each 4-block word
-            mma_mxf4(tmem + kAccCol, da + 2u * j, db + 2u * j, mma_idesc(sf), (tmem + kSfaXCol) | (sf << 30),
-                     (tmem + kSfbCol) | (sf << 30), (kt | j) != 0 ? 1u : 0u);
+          for (uint32_t a = 0; a < 2; ++a) {
+            tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfaXCol + 4 * a, scale_desc(st + L::kOffSfaX + 512 * a));
+            if (kResidual)
+              tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfaRCol + 4 * a, scale_desc(st + L::kOffSfaR + 512 * a));
+            tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfbCol + 8 * a, scale_desc(st + L::kOffSfb + 512 * a));
+            tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfbCol + 8 * a + 4, scale_desc(st + L::kOffSfb + 1024 + 512 * a));
+          }
+          const uint64_t da = operand_desc(st + L::kOffA);
+          const uint64_t db = operand_desc(st + L::kOffB);
+          // 4 MMAs of K = 64 per operand: step q uses k-atom q/2 and scale bytes 2(q%2), 2(q%2)+1.
+#pragma unroll
+          for (uint32_t q = 0; q < 4; ++q) {
+            const uint32_t id = 2u * (q & 1u), a = q >> 1;
+            mma_mxf4_g<kPair>(tmem + kAccCol, da + 2u * q, db + 2u * q, mma_idesc<kPair>(id),
+                              (sf + kSfaXCol + 4 * a) | (id << 30), (sf + kSfbCol + 8 * a) | (id << 30),
+                              (kt | q) != 0 ? 1u : 0u);
           }
           if (kResidual) {
-            const uint64_t dr = operand_desc(st + kOffR);
+            const uint64_t dr = operand_desc(st + L::kOffR);
 #pragma unroll
-            for (uint32_t j = 0; j < 2; ++j) {
-              const uint32_t sf = 2u * j;
-              mma_mxf4(tmem + kAccCol, dr + 2u * j, db + 2u * j, mma_idesc(sf), (tmem + kSfaRCol) | (sf << 30),
-                       (tmem + kSfbCol) | (sf << 30), 1u);
+            for (uint32_t q = 0; q < 4; ++q) {
+              const uint32_t id = 2u * (q & 1u), a = q >> 1;
+              mma_mxf4_g<kPair>(tmem + kAccCol, dr + 2u * q, db + 2u * q, mma_idesc<kPair>(id),
+                                (sf + kSfaRCol + 4 * a) | (id << 30), (sf + kSfbCol + 8 * a) | (id << 30), 1u);
             }
           }
-          tc_commit(&empty[stage]);
-          if (++stage == kStages) {
+          tc_commit_g<kPair>(&empty[stage]);
+          if (++stage == static_cast<uint32_t>(L::kStages)) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(acc_full);
+        tc_commit_g<kPair>(acc_full);
         acc_phase ^= 1u;
       }
       if (!ok) {
         // Teardown after an abort: wait for the MMAs already issued.
-        tc_commit(drain);
+        tc_commit_g<kPair>(drain);
         int never = 0;
         mbar_wait(drain, 0, &never, &g_device_error, kErrWaitDrain);
       }
@@ -265,8 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // at once, so converting and storing Y overlaps the next tile's mainloop.
     const int quad = warp & 3;                // TMEM lanes this warp may access: 32*quad .. 32*quad+31
     const int half = (warp - 2) >> 2;         // columns [128*half, 128*half + 128)
+    const uint32_t acc_empty_leader = kPair == 2 ? map_to_cta(smem_addr(acc_empty), 0) : 0u;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+    for (int tile = unit; tile < p.num_tiles; tile += num_units) {
       const int mb = tile / p.num_nb;
       const int nb = tile - mb * p.num_nb;
       if (!mbar_wait(acc_full, acc_phase, abort_flag, &g_device_error, kErrWaitAccFull)) break;
@@ -278,10 +325,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
+      if (lane == 0) {
+        if constexpr (kPair == 2) mbar_arrive_remote(acc_empty_leader);
+        else mbar_arrive(acc_empty);
+      }
       acc_phase ^= 1u;
 
-      const int row = mb * kBM + quad * 32 + lane;
+      const int row = (mb * kPair + static_cast<int>(rank)) * kBM + quad * 32 + lane;
       const int col0 = nb * kBN + half * 128;
       if (row < p.M) {
         if (kBf16Out) {
@@ -315,11 +365,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  if (kPair == 2) cluster_sync();   // neither CTA leaves while the pair's MMAs or copies may touch it
+  else __syncthreads();
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc_g<kPair>(tmem, kTmemCols);
   }
 }
 
@@ -327,28 +378,71 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-// 2-D map over packed codes [rows][K/2] bytes; box = 64 bytes x box_rows rows,
-// 64-byte swizzle (the layout operand_desc() describes), zero fill outside.
+// 2-D map over packed codes [rows][K/2] bytes; box = 128 bytes x box_rows rows,
+// 128-byte swizzle (the layout operand_desc() describes), zero fill outside.
 bool encode_codes_map(EncodeTiledFn encode, CUtensorMap* map, const void* codes, int64_t rows, int64_t K,
                       uint32_t box_rows) {
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(kBKBytes), box_rows};
   cuuint32_t elem_strides[2] = {1, 1};
-  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box,
-                      elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box, elem_strides,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool kResidual, bool kBf16Out>
-cudaError_t launch_typed(const CUtensorMap& tx, const CUtensorMap& tr, const CUtensorMap& tw, const GemmParams& p,
-                         int grid, cudaStream_t stream) {
-  auto kernel = rfq_gemm_kernel<kResidual, kBf16Out>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+// 4-D map over a scale array in the MMA layout: [row tiles][k atoms][2][256 B]
+// (a 512-byte atom = 128 rows x 4 blocks = 128 K).  The box takes 2 consecutive
+// k-atoms (one 256-K stage) of `box_tiles` consecutive row tiles; atoms past the
+// end in either direction read as zeros.
+bool encode_scales_map(EncodeTiledFn encode, CUtensorMap* map, const void* scales, int64_t rows, int64_t K,
+                       uint32_t box_tiles) {
+  const int64_t row_tiles = (rows + 127) / 128;
+  const int64_t k_atoms = (K / 32 + 3) / 4;
+  cuuint64_t dims[4] = {256, 2, static_cast<cuuint64_t>(k_atoms), static_cast<cuuint64_t>(row_tiles)};
+  cuuint64_t strides[3] = {256, 512, static_cast<cuuint64_t>(k_atoms * 512)};
+  cuuint32_t box[4] = {256, 2, 2, box_tiles};
+  cuuint32_t elem_strides[4] = {1, 1, 1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(scales), dims, strides, box, elem_strides,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int kPair, bool kResidual, bool kBf16Out>
+cudaError_t launch_typed(const Maps& maps, const GemmParams& p, int grid, cudaStream_t stream) {
+  auto kernel = rfq_gemm_kernel<kPair, kResidual, kBf16Out>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<kPair>::kSmem);
   if (e != cudaSuccess) return e;
-  kernel<<<grid, kThreads, kSmemBytes, stream>>>(tx, tr, tw, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Layout<kPair>::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kPair;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kernel, maps, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+template <int kPair>
+cudaError_t launch_mode(const Maps& maps, GemmParams p, int64_t M, bool residual, bool y_bf16, int num_sms,
+                        cudaStream_t stream) {
+  const int64_t num_mb = (M + kBM * kPair - 1) / (kBM * kPair);
+  p.num_tiles = static_cast<int>(num_mb * p.num_nb);
+  int units = num_sms / kPair;
+  if (units > p.num_tiles) units = p.num_tiles;
+  const int grid = units * kPair;
+  if (residual)
+    return y_bf16 ? launch_typed<kPair, true, true>(maps, p, grid, stream)
+                  : launch_typed<kPair, true, false>(maps, p, grid, stream);
+  return y_bf16 ? launch_typed<kPair, false, true>(maps, p, grid, stream)
+                : launch_typed<kPair, false, false>(maps, p, grid, stream);
 }
 
 }  // namespace
@@ -358,35 +452,30 @@ cudaError_t launch_gemm(const void* qx_codes, const void* qx_scales, const void*
                         bool y_bf16, int num_sms, void* encode_tiled, int skip_fill, cudaStream_t stream) {
   EncodeTiledFn encode = reinterpret_cast<EncodeTiledFn>(encode_tiled);
   const bool residual = qr_codes != nullptr;
-  CUtensorMap tx, tr, tw;
-  if (!encode_codes_map(encode, &tx, qx_codes, M, K, kBM)) return cudaErrorInvalidValue;
-  if (!encode_codes_map(encode, &tw, qw_codes, N, K, kBN)) return cudaErrorInvalidValue;
+  // CTA pairs once there are rows for both CTAs of a pair; single CTAs for short M.
+  const bool pair = M > kBM;
+  Maps maps;
+  if (!encode_codes_map(encode, &maps.x, qx_codes, M, K, kBM)) return cudaErrorInvalidValue;
+  if (!encode_codes_map(encode, &maps.w, qw_codes, N, K, pair ? kBN / 2 : kBN)) return cudaErrorInvalidValue;
+  if (!encode_scales_map(encode, &maps.sx, qx_scales, M, K, 1)) return cudaErrorInvalidValue;
+  if (!encode_scales_map(encode, &maps.sw, qw_scales, N, K, 2)) return cudaErrorInvalidValue;
   if (residual) {
-    if (!encode_codes_map(encode, &tr, qr_codes, M, K, kBM)) return cudaErrorInvalidValue;
+    if (!encode_codes_map(encode, &maps.r, qr_codes, M, K, kBM)) return cudaErrorInvalidValue;
+    if (!encode_scales_map(encode, &maps.sr, qr_scales, M, K, 1)) return cudaErrorInvalidValue;
   } else {
-    tr = tx;
+    maps.r = maps.x;
+    maps.sr = maps.sx;
   }
   GemmParams p;
-  p.sfa_x = static_cast<const uint8_t*>(qx_scales);
-  p.sfa_r = static_cast<const uint8_t*>(qr_scales);
-  p.sfb = static_cast<const uint8_t*>(qw_scales);
   p.y = y;
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.num_kt = static_cast<int>((K + kBK - 1) / kBK);
-  p.atoms_per_rowtile = p.num_kt;
-  const int64_t num_mb = (M + kBM - 1) / kBM;
   p.num_nb = static_cast<int>((N + kBN - 1) / kBN);
-  p.num_tiles = static_cast<int>(num_mb * p.num_nb);
-  p.b_rowtiles = static_cast<int>((N + 127) / 128);
+  p.num_tiles = 0;
   p.skip_fill = skip_fill;
-  const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-  if (residual) {
-    return y_bf16 ? launch_typed<true, true>(tx, tr, tw, p, grid, stream)
-                  : launch_typed<true, false>(tx, tr, tw, p, grid, stream);
-  }
-  return y_bf16 ? launch_typed<false, true>(tx, tr, tw, p, grid, stream)
-                : launch_typed<false, false>(tx, tr, tw, p, grid, stream);
+  return pair ? launch_mode<2>(maps, p, M, residual, y_bf16, num_sms, stream)
+              : launch_mode<1>(maps, p, M, residual, y_bf16, num_sms, stream);
 }
 
 cudaError_t read_and_clear_device_error(unsigned int* value) {
