@@ -5,8 +5,8 @@ A step is one pass of the whole hot path on the LLM FFN up-projection workload
   1. rfq_quantize_weight   W -> Q(W)                       (kernel 1, no residual)
   2. rfq_quantize_mxfp4    X -> Q(X), Q(R), R = X - DQ(Q(X)) (kernel 1, fused)
   3. rfq_gemm              Y = DQ(QX) DQ(QW)^T + DQ(QR) DQ(QW)^T (kernel 2, tcgen05)
-Inputs are resident in HBM; L2 is flushed (256 MiB write) between timed steps,
-outside the per-step CUDA events.  ``value`` is executed MMA TFLOP/s over the
+Inputs are resident in HBM; L2 is flushed between timed steps (a 256 MiB buffer
+is written, then read back so L2 is left clean), outside the per-step CUDA events.  ``value`` is executed MMA TFLOP/s over the
 whole step (4*M*N*K per step: the residual doubles K on the tensor pipe).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--all-configs]
@@ -30,6 +30,18 @@ sys.path.insert(0, ROOT)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense MXFP4 : bf16 tensor throughput on B200
 L2_FLUSH_BYTES = 256 << 20
+
+
+def make_l2_flush(torch):
+    """Flush L2 between timed launches: write a 256 MiB buffer (twice L2), then read it
+    back so that L2 holds clean lines and the next timed kernel pays no write-back of
+    the flush itself."""
+    buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def flush():
+        buf.zero_()
+        buf.sum(dtype=torch.int64)
+    return flush
 
 
 def load_peaks():
@@ -235,8 +247,7 @@ def run_cuda(args, rank, world, local):
     peaks = load_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     hbm_peak = peaks["hbm_gbs"]
-    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    flush = lambda: flush_buf.zero_()
+    flush = make_l2_flush(torch)
 
     wk = wl.ffn_up(seed=rank)
     M, K, N = wk.M, wk.K, wk.N
@@ -349,7 +360,7 @@ def run_cuda(args, rank, world, local):
         "data": "synthetic (seeded numpy: N(0,1) + 0.5% outlier channels x50 + 0.01% spikes x500; W N(0,0.02))",
         "config": {"workload": wk.name, "M": M, "K": K, "N": N, "rfq": True, "y": "bf16",
                    "step": "rfq_quantize_weight + rfq_quantize_mxfp4 (X, residual) + rfq_gemm",
-                   "l2": "flushed between steps (256 MiB write, outside the step events)",
+                   "l2": "flushed between steps (256 MiB written then read back, outside the step events)",
                    "parallelism": f"replicas x{world}"},
         "gemm": {"ms": gemm_ms, "tflops_executed": gemm_tflops, "tflops_useful": gemm_tflops / 2,
                  "frac_fp4_peak": gemm_tflops / fp4_peak},
@@ -456,8 +467,7 @@ def run_single_kernel(args):
     step.quantize_w()
     step.quantize_x()
     fn = {"quantize": step.quantize_x, "gemm": step.gemm, "linear": step.run}[args.kernel]
-    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    t = time_kernel(fn, args.steps, lambda: flush_buf.zero_())
+    t = time_kernel(fn, args.steps, make_l2_flush(torch))
     rfq.check_device_error()
     ms = statistics.mean(t)
     out = {"kernel": args.kernel, "M": M, "K": K, "N": N, "rfq": not args.no_rfq, "iters": args.steps,

@@ -39,13 +39,13 @@ def _deps(src: str):
     return [src] + heads + [os.path.join(INCLUDE, "rfq.h")]
 
 
-def _compile(src_name: str, verbose_ptxas: bool) -> str:
+def _compile(src_name: str, verbose_ptxas: bool, build_dir: str = BUILD_DIR, extra_flags=()) -> str:
     src = os.path.join(CSRC, src_name)
-    obj = os.path.join(BUILD_DIR, src_name.replace(".cu", ".o"))
+    obj = os.path.join(build_dir, src_name.replace(".cu", ".o"))
     newest = max(os.path.getmtime(d) for d in _deps(src))
-    if os.path.exists(obj) and os.path.getmtime(obj) >= newest and not verbose_ptxas:
+    if os.path.exists(obj) and os.path.getmtime(obj) >= newest and not verbose_ptxas and not extra_flags:
         return obj
-    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -56,24 +56,27 @@ def _compile(src_name: str, verbose_ptxas: bool) -> str:
     return obj
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    """Compile csrc/*.cu for sm_100a and link librfq.so next to this file."""
-    os.makedirs(BUILD_DIR, exist_ok=True)
+def build(force: bool = False, verbose_ptxas: bool = False, out_lib: str = LIB, extra_flags=()) -> str:
+    """Compile csrc/*.cu for sm_100a and link librfq.so next to this file (or to
+    `out_lib`, with `extra_flags` such as -D overrides of the kernels' tuning knobs)."""
+    build_dir = BUILD_DIR if out_lib == LIB else os.path.join(os.path.dirname(out_lib), "_build")
+    os.makedirs(build_dir, exist_ok=True)
     if force:
-        for f in os.listdir(BUILD_DIR):
-            os.remove(os.path.join(BUILD_DIR, f))
+        for f in os.listdir(build_dir):
+            os.remove(os.path.join(build_dir, f))
     with ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas), SOURCES))
-    if (not force and os.path.exists(LIB)
-            and os.path.getmtime(LIB) >= max(os.path.getmtime(o) for o in objs)):
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas, build_dir, tuple(extra_flags)), SOURCES))
+    if (not force and not extra_flags and os.path.exists(out_lib)
+            and os.path.getmtime(out_lib) >= max(os.path.getmtime(o) for o in objs)):
+        return out_lib
+    LIB_ = out_lib
+    tmp = LIB_ + f".tmp{os.getpid()}"
     cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, LIB_)
+    return LIB_
 
 
 if __name__ == "__main__":

@@ -65,12 +65,17 @@ rfq_status_t current_device(int* num_sms) {
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-// Limits: rows and K fit the kernels' 32-bit tile coordinates, and a matrix holds
-// at most 2^31 - 64 blocks of 32 elements (the quantizer's TMA row coordinate,
-// which runs up to 31 blocks past the last one).
+// Limits: rows and K fit the kernels' 32-bit tile coordinates, a matrix holds at
+// most 2^31 - 64 blocks of 32 elements (the quantizer's 32-bit block indices and
+// TMA row coordinate, which runs up to a span past the last block), and a scale
+// array stays below 2^32 bytes (32-bit offsets).
 bool shape_ok(int64_t rows, int64_t K) {
-  return rows >= 0 && K >= 0 && (K % 32) == 0 && rows <= (int64_t(1) << 31) - 1 && K <= (int64_t(1) << 31) - 32 &&
-         (K == 0 || rows <= ((int64_t(1) << 31) - 64) / (K / 32));
+  if (rows < 0 || K < 0 || (K % 32) != 0 || rows > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 31) - 32) return false;
+  if (K == 0) return true;
+  const int64_t kb = K / 32;
+  if (rows > ((int64_t(1) << 31) - 64) / kb) return false;
+  // the scale array (rows padded to 128, blocks to 4) stays below 2^32 bytes
+  return (rows + 127) / 128 * 128 * ((kb + 3) / 4 * 4) < (int64_t(1) << 32);
 }
 
 rfq_status_t check_quantize_args(const void* x, int64_t M, int64_t K, const void* qc, const void* qs, const void* rc,

@@ -38,25 +38,41 @@ __device__ unsigned int g_quant_error = 0;
 
 namespace {
 
-constexpr int kWarps = 8;
+// Launch shape and ring (compile-time; the defaults are the tuned configuration).
+#ifndef RFQ_Q_STAGES
+#define RFQ_Q_STAGES 4
+#endif
+#ifndef RFQ_Q_SUB
+#define RFQ_Q_SUB 1
+#endif
+#ifndef RFQ_Q_WARPS
+#define RFQ_Q_WARPS 8
+#endif
+#ifndef RFQ_Q_CTAS_PER_SM
+#define RFQ_Q_CTAS_PER_SM 2
+#endif
+constexpr int kWarps = RFQ_Q_WARPS;
 constexpr int kThreads = kWarps * 32;
-constexpr int kStages = 4;
-constexpr int kSpanBlocks = 32;                  // one block per lane
-constexpr int kSpanBytes = kSpanBlocks * 64;     // 2 KiB
+constexpr int kStages = RFQ_Q_STAGES;            // spans in flight per warp
+constexpr int kSub = RFQ_Q_SUB;                  // blocks per lane per span
+constexpr int kSpanBlocks = 32 * kSub;
+constexpr int kSpanBytes = kSpanBlocks * 64;
 constexpr unsigned int kErrQuantWait = 6;        // a warp's wait for its TMA span ran out
 constexpr uint32_t kSmemBytes = kWarps * kStages * kSpanBytes + kWarps * kStages * 8 + 1024;
 
+// Indices are 32-bit: the C ABI limits a matrix to fewer than 2^31 blocks and
+// its scale array to fewer than 2^32 bytes.
 struct QuantParams {
   uint8_t* qx_codes;
   uint8_t* qx_scales;
   uint8_t* qr_codes;
   uint8_t* qr_scales;
-  int64_t M;             // rows
-  int64_t Kb;            // 32-element blocks per row
-  int64_t kb4_per_tile;  // 4-block words per row in the scale layout = ceil(Kb / 4)
-  int64_t rows_pad;      // ceil(M / 128) * 128
-  int64_t total_blocks;  // M * Kb
-  int64_t num_spans;     // ceil(total_blocks / 32)
+  uint32_t M;             // rows
+  uint32_t Kb;            // 32-element blocks per row
+  uint32_t kb4_per_tile;  // 4-block words per row in the scale layout = ceil(Kb / 4)
+  uint32_t rows_pad;      // ceil(M / 128) * 128
+  uint32_t total_blocks;  // M * Kb
+  uint32_t num_spans;     // ceil(total_blocks / span)
 };
 
 // ---------------------------------------------------------------- arithmetic helpers
@@ -103,6 +119,12 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
+// bf16 pair word -> the two fp32 values (element 2j from the low half; exact).
+__device__ __forceinline__ void unpack_bf16x2(uint32_t w, float& lo, float& hi) {
+  lo = __uint_as_float(w << 16);
+  hi = __uint_as_float(w & 0xffff0000u);
+}
+
 // One word of 8 E2M1 codes -> their exact values as fp32.  The magnitudes
 // {0, .5, 1, 1.5, 2, 3, 4, 6} are bf16 0x0000, 0x3F00, 0x3F80, 0x3FC0, 0x4000,
 // 0x4040, 0x4080, 0x40C0: two 8-entry byte tables (high and low bytes) indexed by
@@ -120,8 +142,7 @@ __device__ __forceinline__ void decode8(uint32_t cw, const uint32_t* xw, float* 
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t bf2 = pr[j] | (xw[j] & 0x80008000u);
-    v[2 * j] = __uint_as_float(bf2 << 16);
-    v[2 * j + 1] = __uint_as_float(bf2 & 0xffff0000u);
+    unpack_bf16x2(bf2, v[2 * j], v[2 * j + 1]);
   }
 }
 
@@ -148,27 +169,30 @@ __device__ __forceinline__ float scale_value(uint32_t s) {
 // Byte offset in the MMA scale layout of (row r, 4-block word kb4): atoms of 128
 // rows x 4 blocks with the block-tile index fastest; row r inside its atom at
 // (r % 32) * 16 + ((r / 32) % 4) * 4.
-__device__ __forceinline__ int64_t scale_word_offset(int64_t r, int64_t kb4, int64_t kb4_per_tile) {
-  return ((r >> 7) * kb4_per_tile + kb4) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4;
+__device__ __forceinline__ uint32_t scale_word_offset(uint32_t r, uint32_t kb4, uint32_t kb4_per_tile) {
+  return ((r >> 7) * kb4_per_tile + kb4) * 512u + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u;
 }
 
 // Store one block's scale byte: as a gathered 32-bit word of 4 lanes (word mode)
 // or as a byte.  Called by all 32 lanes (the gather shuffles).
 template <bool kWordScales>
-__device__ __forceinline__ void store_scale(uint8_t* scales, uint32_t s, bool valid, int64_t row, int64_t kb,
-                                            int64_t kb4_per_tile, int lane) {
+__device__ __forceinline__ void store_scale(uint8_t* scales, uint32_t s, bool valid, uint32_t row, uint32_t kb,
+                                            uint32_t kb4_per_tile, int lane) {
   if constexpr (kWordScales) {
-    const int base = lane & ~3;
-    const uint32_t w = __shfl_sync(0xffffffffu, s, base) | (__shfl_sync(0xffffffffu, s, base + 1) << 8) |
-                       (__shfl_sync(0xffffffffu, s, base + 2) << 16) | (__shfl_sync(0xffffffffu, s, base + 3) << 24);
+    // lanes 4j..4j+3 hold blocks 4j..4j+3: two shuffles pack them into lane 4j's word
+    const uint32_t s01 = s | (__shfl_down_sync(0xffffffffu, s, 1) << 8);
+    const uint32_t w = s01 | (__shfl_down_sync(0xffffffffu, s01, 2) << 16);
     if (valid && (lane & 3) == 0) *reinterpret_cast<uint32_t*>(scales + scale_word_offset(row, kb >> 2, kb4_per_tile)) = w;
   } else {
     if (valid) scales[scale_word_offset(row, kb >> 2, kb4_per_tile) + (kb & 3)] = static_cast<uint8_t>(s);
   }
 }
 
-template <bool kResidual, bool kWordScales>
-__global__ void __launch_bounds__(kThreads, 2)
+// kWide: X seen as [blocks/2][128 bytes] with a 128-byte swizzle (needs an even
+// block count); otherwise as [blocks][64 bytes] with a 64-byte swizzle.  Either
+// way a lane's four 16-byte reads of its block hit distinct banks.
+template <bool kResidual, bool kWordScales, bool kWide>
+__global__ void __launch_bounds__(kThreads, RFQ_Q_CTAS_PER_SM)
     rfq_quantize_kernel(const __grid_constant__ CUtensorMap tm_x, const QuantParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -178,64 +202,70 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kStages * kSpanBytes) + warp * kStages;
   volatile int abort_flag = 0;   // per warp: each warp's ring is independent
 
-  const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
-  const int64_t GW = static_cast<int64_t>(gridDim.x) * kWarps;
-  const int64_t n_my = p.num_spans > gw ? (p.num_spans - gw + GW - 1) / GW : 0;
+  const uint32_t gw = blockIdx.x * kWarps + warp;
+  const uint32_t GW = gridDim.x * kWarps;
+  const uint32_t n_my = p.num_spans > gw ? (p.num_spans - gw + GW - 1) / GW : 0;
+  // TMA row coordinate of a span: rows of 128 bytes (2 blocks) or of 64 bytes (1 block)
+  auto span_row = [&](uint32_t span) { return static_cast<int>(span * (kWide ? kSpanBlocks / 2 : kSpanBlocks)); };
 
   if (lane == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+    for (int st = 0; st < kStages; ++st) mbar_init(&bars[st], 1);
     fence_mbar_init();
-    for (int s = 0; s < kStages && s < n_my; ++s) {
-      mbar_arrive_expect_tx(&bars[s], kSpanBytes);
-      tma_load_2d(ring + s * kSpanBytes, &tm_x, &bars[s], 0, static_cast<int>((gw + s * GW) * kSpanBlocks));
+    for (uint32_t st = 0; st < kStages && st < n_my; ++st) {
+      mbar_arrive_expect_tx(&bars[st], kSpanBytes);
+      tma_load_2d(ring + st * kSpanBytes, &tm_x, &bars[st], 0, span_row(gw + st * GW));
     }
   }
   __syncwarp();
 
-  // Block coordinates of lane 0's block, advanced incrementally span by span.
-  const int64_t stride_blocks = GW * kSpanBlocks;
-  const int64_t d_row = stride_blocks / p.Kb, d_kb = stride_blocks - (stride_blocks / p.Kb) * p.Kb;
-  int64_t row0 = (gw * kSpanBlocks) / p.Kb;
-  int64_t kb0 = gw * kSpanBlocks - row0 * p.Kb;
-  const int swz = (lane >> 1) & 3;   // 64-byte swizzle of this lane's row in the span
+  // Block coordinates of the span's first block, advanced incrementally span by span.
+  const uint32_t stride_blocks = GW * kSpanBlocks;
+  const uint32_t d_row = stride_blocks / p.Kb, d_kb = stride_blocks - d_row * p.Kb;
+  uint32_t row0 = (gw * kSpanBlocks) / p.Kb;
+  uint32_t kb0 = gw * kSpanBlocks - row0 * p.Kb;
+  // Byte offset of this lane's block inside a 32-block sub-span, and the swizzle of its row.
+  const int lane_off = kWide ? (lane >> 1) * 128 + (lane & 1) * 64 : lane * 64;
+  const int swz = kWide ? (lane >> 1) & 7 : (lane >> 1) & 3;
 
-  int64_t i = 0;
+  uint32_t i = 0;
   for (; i < n_my; ++i) {
     const int s = static_cast<int>(i % kStages);
-    const bool ok = mbar_wait(&bars[s], static_cast<uint32_t>((i / kStages) & 1), &abort_flag, &g_quant_error,
-                              kErrQuantWait);
+    const bool ok = mbar_wait(&bars[s], (i / kStages) & 1u, &abort_flag, &g_quant_error, kErrQuantWait);
     if (!__all_sync(0xffffffffu, ok)) break;   // every lane returns from its bounded wait: a uniform decision
-    const int64_t gb = (gw + i * GW) * kSpanBlocks + lane;
+
+#pragma unroll 1
+    for (int u = 0; u < kSub; ++u) {
+    const uint32_t gb = (gw + i * GW) * kSpanBlocks + u * 32 + lane;
     const bool valid = gb < p.total_blocks;
     // lane's block: row, block-in-row
-    int64_t row, kb;
+    uint32_t row, kb;
     {
-      const int64_t t = kb0 + lane;
-      int64_t q;
-      if (p.Kb >= kSpanBlocks) q = t >= p.Kb ? 1 : 0;
-      else q = static_cast<int64_t>(static_cast<uint32_t>(t) / static_cast<uint32_t>(p.Kb));
+      const uint32_t t = kb0 + u * 32 + lane;
+      const uint32_t q = p.Kb >= kSpanBlocks ? (t >= p.Kb ? 1u : 0u) : t / p.Kb;
       row = row0 + q;
       kb = t - q * p.Kb;
     }
 
     uint32_t w[16];
-    const uint8_t* src = ring + s * kSpanBytes + lane * 64;
+    const uint8_t* src = ring + s * kSpanBytes + u * 2048 + lane_off;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint4 c = *reinterpret_cast<const uint4*>(src + ((j ^ swz) << 4));
+      const int chunk = kWide ? (((lane & 1) * 4 + j) ^ swz) - (lane & 1) * 4 : (j ^ swz);
+      const uint4 c = *reinterpret_cast<const uint4*>(src + chunk * 16);
       w[4 * j + 0] = c.x;
       w[4 * j + 1] = c.y;
       w[4 * j + 2] = c.z;
       w[4 * j + 3] = c.w;
     }
-    __syncwarp();
-    // This lane's data are now in registers: refill the stage with the span
-    // kStages ahead (the reads above are ordered before the async-proxy write).
-    if (lane == 0 && i + kStages < n_my) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive_expect_tx(&bars[s], kSpanBytes);
-      tma_load_2d(ring + s * kSpanBytes, &tm_x, &bars[s], 0,
-                  static_cast<int>((gw + (i + kStages) * GW) * kSpanBlocks));
+    if (u == kSub - 1) {
+      __syncwarp();
+      // This warp's data are now in registers: refill the stage with the span
+      // kStages ahead (the reads above are ordered before the async-proxy write).
+      if (lane == 0 && i + kStages < n_my) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive_expect_tx(&bars[s], kSpanBytes);
+        tma_load_2d(ring + s * kSpanBytes, &tm_x, &bars[s], 0, span_row(gw + (i + kStages) * GW));
+      }
     }
 
     // ---- Q(X): block amax on bf16 magnitudes (NaN-propagating), E8M0 byte
@@ -261,8 +291,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       float xv[8], v[8];
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        xv[2 * h] = __uint_as_float(w[4 * k + h] << 16);
-        xv[2 * h + 1] = __uint_as_float(w[4 * k + h] & 0xffff0000u);
+        unpack_bf16x2(w[4 * k + h], xv[2 * h], xv[2 * h + 1]);
         mul2(v[2 * h], v[2 * h + 1], xv[2 * h], xv[2 * h + 1], inv_x);
       }
       cx[k] = encode8(v);
@@ -278,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
     }
-    if (valid) *reinterpret_cast<uint4*>(p.qx_codes + gb * 16) = make_uint4(cx[0], cx[1], cx[2], cx[3]);
+    if (valid) *reinterpret_cast<uint4*>(p.qx_codes + static_cast<size_t>(gb) * 16) = make_uint4(cx[0], cx[1], cx[2], cx[3]);
     store_scale<kWordScales>(p.qx_scales, sx, valid, row, kb, p.kb4_per_tile, lane);
 
     if constexpr (kResidual) {
@@ -294,9 +323,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int h = 0; h < 4; ++h) mul2(v[2 * h], v[2 * h + 1], r[8 * k + 2 * h], r[8 * k + 2 * h + 1], inv_r);
         cr[k] = encode8(v);
       }
-      if (valid) *reinterpret_cast<uint4*>(p.qr_codes + gb * 16) = make_uint4(cr[0], cr[1], cr[2], cr[3]);
+      if (valid) *reinterpret_cast<uint4*>(p.qr_codes + static_cast<size_t>(gb) * 16) = make_uint4(cr[0], cr[1], cr[2], cr[3]);
       store_scale<kWordScales>(p.qr_scales, sr, valid, row, kb, p.kb4_per_tile, lane);
     }
+
+    }  // sub-spans
 
     kb0 += d_kb;
     row0 += d_row;
@@ -309,26 +340,25 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (i < n_my && lane == 0) {
     // A wait ran out: let this warp's outstanding copies land before leaving.
     int never = 0;
-    for (int64_t k = i; k < n_my && k < i + kStages; ++k)
+    for (uint32_t k = i; k < n_my && k < i + kStages; ++k)
       mbar_wait(&bars[k % kStages], static_cast<uint32_t>((k / kStages) & 1), &never, &g_quant_error, kErrQuantWait);
   }
 
   // ---- zero padding of the scale arrays: rows [M, rows_pad) and blocks [Kb, 4*kb4) of real rows
-  const int64_t tid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
-  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
-  const int64_t pad_rows = p.rows_pad - p.M;
-  const int64_t pad_words = pad_rows * p.kb4_per_tile;
-  for (int64_t t = tid; t < pad_words; t += nthreads) {
-    const int64_t r = p.M + t / p.kb4_per_tile, kb4 = t % p.kb4_per_tile;
-    const int64_t off = scale_word_offset(r, kb4, p.kb4_per_tile);
+  const uint32_t tid = blockIdx.x * kThreads + threadIdx.x;
+  const uint32_t nthreads = gridDim.x * kThreads;
+  const uint32_t pad_words = (p.rows_pad - p.M) * p.kb4_per_tile;
+  for (uint32_t t = tid; t < pad_words; t += nthreads) {
+    const uint32_t r = p.M + t / p.kb4_per_tile, kb4 = t % p.kb4_per_tile;
+    const uint32_t off = scale_word_offset(r, kb4, p.kb4_per_tile);
     *reinterpret_cast<uint32_t*>(p.qx_scales + off) = 0u;
     if (kResidual) *reinterpret_cast<uint32_t*>(p.qr_scales + off) = 0u;
   }
-  const int64_t tail = p.kb4_per_tile * 4 - p.Kb;   // 0..3 pad blocks per real row
+  const uint32_t tail = p.kb4_per_tile * 4 - p.Kb;   // 0..3 pad blocks per real row
   if (tail > 0) {
-    for (int64_t t = tid; t < p.M * tail; t += nthreads) {
-      const int64_t r = t / tail, kb = p.Kb + t % tail;
-      const int64_t off = scale_word_offset(r, kb >> 2, p.kb4_per_tile) + (kb & 3);
+    for (uint32_t t = tid; t < p.M * tail; t += nthreads) {
+      const uint32_t r = t / tail, kb = p.Kb + t % tail;
+      const uint32_t off = scale_word_offset(r, kb >> 2, p.kb4_per_tile) + (kb & 3);
       p.qx_scales[off] = 0;
       if (kResidual) p.qr_scales[off] = 0;
     }
@@ -339,13 +369,23 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-template <bool kResidual, bool kWord>
+#ifndef RFQ_Q_WIDE
+#define RFQ_Q_WIDE 1
+#endif
+
+template <bool kResidual, bool kWord, bool kWide>
 cudaError_t launch_typed(const CUtensorMap& tm, const QuantParams& p, int grid, cudaStream_t stream) {
-  auto kernel = rfq_quantize_kernel<kResidual, kWord>;
+  auto kernel = rfq_quantize_kernel<kResidual, kWord, kWide>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm, p);
   return cudaGetLastError();
+}
+
+template <bool kResidual, bool kWord>
+cudaError_t launch_width(bool wide, const CUtensorMap& tm, const QuantParams& p, int grid, cudaStream_t stream) {
+  return wide ? launch_typed<kResidual, kWord, true>(tm, p, grid, stream)
+              : launch_typed<kResidual, kWord, false>(tm, p, grid, stream);
 }
 
 }  // namespace
@@ -357,37 +397,38 @@ cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, void* qx_codes,
   p.qx_scales = static_cast<uint8_t*>(qx_scales);
   p.qr_codes = static_cast<uint8_t*>(qr_codes);
   p.qr_scales = static_cast<uint8_t*>(qr_scales);
-  p.M = M;
-  p.Kb = K / 32;
+  p.M = static_cast<uint32_t>(M);
+  p.Kb = static_cast<uint32_t>(K / 32);
   p.kb4_per_tile = (p.Kb + 3) / 4;
-  p.rows_pad = (M + 127) / 128 * 128;
-  p.total_blocks = M * p.Kb;
+  p.rows_pad = static_cast<uint32_t>((M + 127) / 128 * 128);
+  p.total_blocks = static_cast<uint32_t>(M * (K / 32));
   p.num_spans = (p.total_blocks + kSpanBlocks - 1) / kSpanBlocks;
 
-  // X as [total_blocks][64 bytes]; 32-row boxes, 64-byte swizzle, zero fill past the end.
+  // X as [total_blocks/2][128 bytes] (128-byte swizzle) when the block count is
+  // even, else as [total_blocks][64 bytes] (64-byte swizzle); boxes of one span;
+  // zero fill past the end.
+  const bool wide = RFQ_Q_WIDE && (p.total_blocks % 2) == 0;
   CUtensorMap tm;
-  cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(p.total_blocks)};
-  cuuint64_t strides[1] = {64};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kSpanBlocks)};
+  cuuint64_t dims[2] = {wide ? 128u : 64u, static_cast<cuuint64_t>(wide ? p.total_blocks / 2 : p.total_blocks)};
+  cuuint64_t strides[1] = {wide ? 128u : 64u};
+  cuuint32_t box[2] = {wide ? 128u : 64u, static_cast<cuuint32_t>(wide ? kSpanBlocks / 2 : kSpanBlocks)};
   cuuint32_t elem_strides[2] = {1, 1};
   EncodeTiledFn encode = reinterpret_cast<EncodeTiledFn>(encode_tiled);
   if (encode(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(x), dims, strides, box, elem_strides,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+             CU_TENSOR_MAP_INTERLEAVE_NONE, wide ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
 
   const int64_t warps_needed = p.num_spans;
   int64_t grid = (warps_needed + kWarps - 1) / kWarps;
-  const int64_t cap = static_cast<int64_t>(num_sms) * 2;
+  const int64_t cap = static_cast<int64_t>(num_sms) * RFQ_Q_CTAS_PER_SM;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   const bool word = (p.Kb % 4) == 0;
-  if (qr_codes) {
-    return word ? launch_typed<true, true>(tm, p, static_cast<int>(grid), stream)
-                : launch_typed<true, false>(tm, p, static_cast<int>(grid), stream);
-  }
-  return word ? launch_typed<false, true>(tm, p, static_cast<int>(grid), stream)
-              : launch_typed<false, false>(tm, p, static_cast<int>(grid), stream);
+  const int g = static_cast<int>(grid);
+  if (qr_codes)
+    return word ? launch_width<true, true>(wide, tm, p, g, stream) : launch_width<true, false>(wide, tm, p, g, stream);
+  return word ? launch_width<false, true>(wide, tm, p, g, stream) : launch_width<false, false>(wide, tm, p, g, stream);
 }
 
 cudaError_t read_and_clear_quant_error(unsigned int* value) {
