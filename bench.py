@@ -144,13 +144,8 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
-    if world == 1:
-        return v
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from block_scaled_gemm_rfq_b200.sharding import max_over_ranks as _max
+    return _max(v) if world > 1 else v
 
 
 # ----------------------------------------------------------------------------- the CUDA path

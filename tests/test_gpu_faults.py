@@ -1,0 +1,44 @@
+"""Failure detection without a GPU fault: every spin-wait inside the GEMM is bounded.
+
+The library's test hook makes the producer of the first CTA skip one stage fill, so
+the MMA warp's wait for that stage runs out (after about 1.5 s).  The kernel then
+records the wait in the device error word, drains its own copies and MMAs, frees its
+TMEM and returns; rfq_check_device_error reports RFQ_ERR_TIMEOUT with detail 1 (the
+stage wait) and the context stays usable: the next GEMM is correct.  Both the
+single-CTA path (M <= 128) and the CTA-pair path (M > 128) are exercised.
+"""
+import numpy as np
+import pytest
+
+from block_scaled_gemm_rfq_b200 import workloads as wl
+from helpers import assert_y_close, dev_bf16, y_to_numpy
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("M", [128, 384])
+def test_skipped_fill_times_out_and_context_survives(rfq, oracle, M):
+    import torch
+    N, K = 256, 1024
+    x_bits = wl.random_matrix(M, K, seed=M, scale=2.0)
+    w_bits = wl.random_matrix(N, K, seed=M + 1, scale=0.05)
+    qa = rfq.quantize_mxfp4_alloc(dev_bf16(x_bits), residual=True)
+    qw = rfq.quantize_weight_alloc(dev_bf16(w_bits))
+    torch.cuda.synchronize()
+    rfq.check_device_error()
+
+    rfq.debug_skip_next_fill(0)
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    rfq.gemm(qa.codes, qa.scales, qa.r_codes, qa.r_scales, qw.codes, qw.scales, M, N, K, y)
+    with pytest.raises(rfq.RFQError) as info:
+        rfq.check_device_error()
+    assert info.value.status == 6          # RFQ_ERR_TIMEOUT
+    assert info.value.detail == 1          # the MMA warp's wait for a loaded stage
+    rfq.check_device_error()               # the error word was cleared
+
+    # the context is still usable and the hook is one-shot
+    y2 = rfq.gemm_alloc(qa, qw, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    rfq.check_device_error()
+    Y, S, _ = oracle.rfq_linear(x_bits, w_bits, residual=True)
+    assert_y_close(y_to_numpy(y2), Y, S, bf16_out=False)
