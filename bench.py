@@ -473,6 +473,48 @@ def run_reference(args):
     }
 
 
+def run_fidelity(args):
+    """--fidelity: the paper's central claim measured on the synthetic workloads with
+    this library's kernels (RFQ paper, abstract and section 1: activation
+    quantization dominates the FP4 error and the residual path recovers it).
+
+    Activation fidelity: a GEMM against the K x K identity (which MXFP4 represents
+    exactly) returns the dequantized activation DQ(QX) [+ DQ(QR)] in fp32, so
+    ||X - X_hat|| / ||X|| is measured with RFQ on and off.  Output fidelity:
+    ||Y - X W^T|| / ||X W^T|| against an fp32 product of the bf16 inputs."""
+    import numpy as np
+    import torch
+
+    import block_scaled_gemm_rfq_b200 as rfq
+    from block_scaled_gemm_rfq_b200 import workloads as wl
+    rfq.load_library()
+    report = {}
+    cases = [("tiny", wl.tiny(0)), ("quantize_bandwidth", wl.quantize_bandwidth(0, M=1024)),
+             ("ffn_up", wl.ffn_up(0, M=1024)), ("dit_ffn", wl.dit_ffn(0, M=1024))]
+    for name, wk in cases:
+        x = to_device_bf16(wk.x_bits)
+        M, K = x.shape
+        eye = torch.eye(K, dtype=torch.bfloat16, device="cuda")
+        qe = rfq.quantize_weight_alloc(eye)
+        xf = x.float()
+        row = {"workload": wk.name, "M": M, "K": K}
+        for res in (True, False):
+            qa = rfq.quantize_mxfp4_alloc(x, residual=res)
+            xhat = rfq.gemm_alloc(qa, qe, out_dtype=torch.float32, use_residual=res)
+            row[f"x_rel_err_{'rfq' if res else 'mxfp4'}"] = float(torch.linalg.norm(xhat - xf) / torch.linalg.norm(xf))
+        if wk.w_bits is not None:
+            w = to_device_bf16(wk.w_bits)
+            yref = xf @ w.float().t()
+            qw = rfq.quantize_weight_alloc(w)
+            for res in (True, False):
+                qa = rfq.quantize_mxfp4_alloc(x, residual=res)
+                y = rfq.gemm_alloc(qa, qw, out_dtype=torch.float32, use_residual=res)
+                row[f"y_rel_err_{'rfq' if res else 'mxfp4'}"] = float(torch.linalg.norm(y - yref) / torch.linalg.norm(yref))
+        rfq.check_device_error()
+        report[name] = row
+    return {"fidelity": report}
+
+
 def run_single_kernel(args):
     """--kernel quantize|gemm|linear: time one kernel on a chosen shape (for sweeps and
     profiles); prints one JSON line with per-launch times."""
@@ -516,12 +558,17 @@ def main():
     ap.add_argument("--N", type=int, default=12288)
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--no-rfq", action="store_true", help="with --kernel: residual path off")
+    ap.add_argument("--fidelity", action="store_true",
+                    help="report activation and output error of RFQ vs plain MXFP4 on the workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
     if args.kernel:
         run_single_kernel(args)
+        return
+    if args.fidelity:
+        print(json.dumps(run_fidelity(args)))
         return
 
     if args.impl == "reference":

@@ -183,9 +183,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  griddep_launch_dependents();
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
+      griddep_wait();   // QX/QR/QW may be written by the previous kernel on the stream
       uint32_t stage = 0, phase = 0;
       uint32_t filled = 0, last_parity = 0;
       int fill = 0;
@@ -418,13 +420,15 @@ cudaError_t launch_typed(const Maps& maps, const GemmParams& p, int grid, cudaSt
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = Layout<kPair>::kSmem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = kPair;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see griddep_wait()
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, kernel, maps, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -180,6 +180,18 @@ __device__ __forceinline__ void tmem_wait_ld() {
 }
 
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Wait until the grids this launch depends on (the previous kernel on the stream)
+// have completed and their memory is visible.  A no-op when the kernel was not
+// launched with programmatic stream serialization.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next kernel on the stream to begin launching (it still waits for this
+// grid to complete before reading what this grid writes).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- clusters and CTA pairs
 __device__ __forceinline__ uint32_t cluster_cta_rank() {
   uint32_t r;

@@ -208,9 +208,11 @@ __global__ void __launch_bounds__(kThreads, RFQ_Q_CTAS_PER_SM)
   // TMA row coordinate of a span: rows of 128 bytes (2 blocks) or of 64 bytes (1 block)
   auto span_row = [&](uint32_t span) { return static_cast<int>(span * (kWide ? kSpanBlocks / 2 : kSpanBlocks)); };
 
+  griddep_launch_dependents();
   if (lane == 0) {
     for (int st = 0; st < kStages; ++st) mbar_init(&bars[st], 1);
     fence_mbar_init();
+    griddep_wait();   // X may be written by the previous kernel on the stream
     for (uint32_t st = 0; st < kStages && st < n_my; ++st) {
       mbar_arrive_expect_tx(&bars[st], kSpanBytes);
       tma_load_2d(ring + st * kSpanBytes, &tm_x, &bars[st], 0, span_row(gw + st * GW));
@@ -345,6 +347,8 @@ __global__ void __launch_bounds__(kThreads, RFQ_Q_CTAS_PER_SM)
   }
 
   // ---- zero padding of the scale arrays: rows [M, rows_pad) and blocks [Kb, 4*kb4) of real rows
+  // (stores to buffers the previous kernel on the stream may still read: wait for it)
+  griddep_wait();
   const uint32_t tid = blockIdx.x * kThreads + threadIdx.x;
   const uint32_t nthreads = gridDim.x * kThreads;
   const uint32_t pad_words = (p.rows_pad - p.M) * p.kb4_per_tile;
@@ -378,7 +382,18 @@ cudaError_t launch_typed(const CUtensorMap& tm, const QuantParams& p, int grid, 
   auto kernel = rfq_quantize_kernel<kResidual, kWord, kWide>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see griddep_wait()
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kernel, tm, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
