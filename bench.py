@@ -232,6 +232,33 @@ def time_kernel(fn, iters, flush):
     return [a.elapsed_time(b) for a, b in out]
 
 
+def time_stream(fns, reps):
+    """Per-call ms of back-to-back calls, replayed from a CUDA graph so that host
+    launch overhead is out of the figure: fns[i] use distinct buffers whose total
+    is larger than L2, so every call reads its operands from HBM.  One pass over
+    all fns is captured; the graph is replayed 3 times untimed, then reps times
+    between one event pair."""
+    import torch
+    for f in fns:   # eager warm-up (first-call setup happens outside the capture)
+        f()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for f in fns:
+            f()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) / (reps * len(fns))
+
+
 def quantize_bytes(M, K, residual):
     """Algorithmic HBM bytes of the fused quantizer: read X once (2 B/elem), write codes
     (0.5 B/elem) and scales (1 B per 32 elements) per output."""
@@ -331,13 +358,39 @@ def run_cuda(args, rank, world, local):
             sk = wl.m_sweep(Ms, seed=rank)
             xs, ws = to_device_bf16(sk.x_bits), to_device_bf16(sk.w_bits)
             row = {}
+            # Layer after layer: distinct weights (and activations) per call, > 2x L2 in total.
+            n_sets = max(2, int(2 * 126e6 // (sk.N * sk.K * 0.53 + Ms * sk.K * 2)) + 1)
             for res in (True, False):
                 qws = rfq.quantize_weight_alloc(ws)
                 y = torch.empty((Ms, sk.N), dtype=torch.bfloat16, device="cuda")
                 wsb = torch.empty(rfq.linear_workspace_bytes(Ms, sk.K, res), dtype=torch.uint8, device="cuda")
                 t = time_kernel(lambda: rfq.linear(xs, qws.codes, qws.scales, sk.N, y, wsb, res), 20, flush)
-                row["rfq" if res else "off"] = {"us": 1e3 * statistics.mean(t),
-                                                "tflops_useful": 2.0 * Ms * sk.N * sk.K / (statistics.mean(t) * 1e-3) / 1e12}
+                sets = [(xs.clone(), rfq.quantize_weight_alloc(ws),
+                         torch.empty((Ms, sk.N), dtype=torch.bfloat16, device="cuda"),
+                         torch.empty(rfq.linear_workspace_bytes(Ms, sk.K, res), dtype=torch.uint8, device="cuda"))
+                        for _ in range(n_sets)]
+                calls = [lambda a=a: rfq.linear(a[0], a[1].codes, a[1].scales, sk.N, a[2], a[3], res) for a in sets]
+                t_stream = time_stream(calls, max(2, 400 // n_sets))
+                cell = {"us": 1e3 * statistics.mean(t),
+                        "tflops_useful": 2.0 * Ms * sk.N * sk.K / (statistics.mean(t) * 1e-3) / 1e12,
+                        "us_stream": 1e3 * t_stream, "stream_sets": n_sets,
+                        "path": "fused" if Ms <= rfq.FUSED_MAX_M else "quantize+gemm"}
+                if Ms <= rfq.FUSED_MAX_M:
+                    # the two-kernel path on the same problem, for comparison
+                    s2 = RfqStep(rfq, xs, ws, residual=res)
+                    s2.quantize_w()
+                    t2 = time_kernel(lambda: (s2.quantize_x(), s2.gemm()), 20, flush)
+                    cell["two_kernel_us"] = 1e3 * statistics.mean(t2)
+                    y2 = torch.empty((Ms, sk.N), dtype=torch.bfloat16, device="cuda")
+
+                    def two(a):
+                        rfq.quantize_mxfp4(a[0], s2.qx_c, s2.qx_s, s2.qr_c, s2.qr_s)
+                        rfq.gemm(s2.qx_c, s2.qx_s, s2.qr_c, s2.qr_s, a[1].codes, a[1].scales, Ms, sk.N, sk.K, y2)
+                    cell["two_kernel_us_stream"] = 1e3 * time_stream([lambda a=a: two(a) for a in sets],
+                                                                     max(2, 400 // n_sets))
+                    del s2
+                del sets
+                row["rfq" if res else "off"] = cell
             sweep[str(Ms)] = row
         extra["m_sweep_rfq_linear"] = sweep
 
@@ -530,11 +583,16 @@ def run_single_kernel(args):
     step = RfqStep(rfq, x, w, residual=not args.no_rfq)
     step.quantize_w()
     step.quantize_x()
-    fn = {"quantize": step.quantize_x, "gemm": step.gemm, "linear": step.run}[args.kernel]
+    fused = lambda: rfq.linear_fused(x, step.qw_c, step.qw_s, N, step.y, not args.no_rfq)
+    fn = {"quantize": step.quantize_x, "gemm": step.gemm, "linear": step.run,
+          "two-kernel": lambda: (step.quantize_x(), step.gemm()), "fused": fused}[args.kernel]
+    rfq.debug_fused_split(args.split)
     t = time_kernel(fn, args.steps, make_l2_flush(torch))
+    rfq.debug_fused_split(0)
     rfq.check_device_error()
     ms = statistics.mean(t)
     out = {"kernel": args.kernel, "M": M, "K": K, "N": N, "rfq": not args.no_rfq, "iters": args.steps,
+           "split": args.split,
            "ms_mean": ms, "ms_min": min(t)}
     if args.kernel == "quantize":
         out["gbs"] = quantize_bytes(M, K, not args.no_rfq) / (ms * 1e-3) / 1e9
@@ -552,8 +610,10 @@ def main():
     ap.add_argument("--all-configs", action="store_true", help="also time the DiT FFN GEMM and the M sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
-    ap.add_argument("--kernel", choices=["quantize", "gemm", "linear"], default=None,
-                    help="time one kernel on --M/--N/--K instead of the benchmark step")
+    ap.add_argument("--kernel", choices=["quantize", "gemm", "linear", "two-kernel", "fused"], default=None,
+                    help="time one kernel on --M/--N/--K instead of the benchmark step (linear = quantize W "
+                         "+ quantize X + GEMM; two-kernel = quantize X + GEMM; fused = rfq_linear_fused)")
+    ap.add_argument("--split", type=int, default=0, help="with --kernel fused: K split (0 = automatic)")
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=12288)
     ap.add_argument("--K", type=int, default=4096)

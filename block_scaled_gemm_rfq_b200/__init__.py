@@ -19,7 +19,8 @@ import threading
 __all__ = [
     "RFQError", "load_library", "library_path", "codes_bytes", "scales_bytes", "linear_workspace_bytes",
     "quantize_mxfp4", "quantize_weight", "gemm", "linear", "linear_static_workspace", "check_device_error",
-    "debug_skip_next_fill", "STATIC_WORKSPACE_BYTES",
+    "debug_skip_next_fill", "STATIC_WORKSPACE_BYTES", "linear_fused", "linear_fused_alloc", "debug_fused_split",
+    "FUSED_MAX_M",
     "QuantizedTensor", "quantize_mxfp4_alloc", "quantize_weight_alloc", "gemm_alloc", "linear_alloc",
     "EXPORTED_SYMBOLS", "OUT_F32", "OUT_BF16",
 ]
@@ -39,11 +40,14 @@ STATUS = {0: "RFQ_OK", 1: "RFQ_ERR_INVALID_ARG", 2: "RFQ_ERR_UNSUPPORTED_SHAPE",
 EXPORTED_SYMBOLS = (
     "rfq_status_string", "rfq_codes_bytes", "rfq_scales_bytes", "rfq_quantize_mxfp4", "rfq_quantize_weight",
     "rfq_gemm", "rfq_linear_workspace_bytes", "rfq_linear", "rfq_check_device_error", "rfq_debug_skip_next_fill",
-    "rfq_linear_static_workspace",
+    "rfq_linear_static_workspace", "rfq_linear_fused", "rfq_debug_fused_split",
 )
 
 # Size of the library's fixed scratch array (RFQ_STATIC_WORKSPACE_BYTES in include/rfq.h).
 STATIC_WORKSPACE_BYTES = 32 << 20
+
+# Largest M of the single-kernel linear layer (RFQ_FUSED_MAX_M in include/rfq.h).
+FUSED_MAX_M = 64
 
 
 class RFQError(RuntimeError):
@@ -78,6 +82,8 @@ def load_library():
                 "rfq_check_device_error": (I, [P, ctypes.POINTER(ctypes.c_int)]),
                 "rfq_debug_skip_next_fill": (I, [I]),
                 "rfq_linear_static_workspace": (I, [P, I64, I64, P, P, I64, P, I, I, P]),
+                "rfq_linear_fused": (I, [P, I64, I64, P, P, I64, P, I, I, P]),
+                "rfq_debug_fused_split": (I, [I]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(lib, name)
@@ -160,6 +166,22 @@ def linear_static_workspace(x, qw_codes, qw_scales, N, y, use_residual=True, str
            "rfq_linear_static_workspace")
 
 
+def linear_fused(x, qw_codes, qw_scales, N, y, use_residual=True, stream=None):
+    """rfq_linear_fused: the RFQ linear layer in one kernel (quantizer inside the GEMM)
+    for M <= FUSED_MAX_M rows; no workspace."""
+    import torch
+    M, K = x.shape
+    y_type = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
+    _check(load_library().rfq_linear_fused(_ptr(x), M, K, _ptr(qw_codes), _ptr(qw_scales), N, _ptr(y), y_type,
+                                           int(bool(use_residual)), _stream(stream)),
+           "rfq_linear_fused")
+
+
+def debug_fused_split(split: int):
+    """Force rfq_linear_fused's split of K over a cluster (1..8); 0 = automatic."""
+    _check(load_library().rfq_debug_fused_split(int(split)), "rfq_debug_fused_split")
+
+
 def check_device_error(stream=None):
     """Synchronize and report a bounded-wait timeout inside a kernel (raises RFQError)."""
     detail = ctypes.c_int(0)
@@ -218,6 +240,14 @@ def gemm_alloc(qa: QuantizedTensor, qw: QuantizedTensor, out_dtype=None, use_res
     res = use_residual and qa.has_residual
     gemm(qa.codes, qa.scales, qa.r_codes if res else None, qa.r_scales if res else None, qw.codes, qw.scales,
          qa.rows, qw.rows, qa.K, y, stream)
+    return y
+
+
+def linear_fused_alloc(x, qw: QuantizedTensor, out_dtype=None, use_residual=True, stream=None):
+    import torch
+    out_dtype = out_dtype or torch.bfloat16
+    y = torch.empty((x.shape[0], qw.rows), dtype=out_dtype, device=x.device)
+    linear_fused(x, qw.codes, qw.scales, qw.rows, y, use_residual, stream)
     return y
 
 

@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "librfq.so")
 BUILD_DIR = os.path.join(PKG, "_build")
 
-SOURCES = ["rfq_api.cu", "rfq_quantize.cu", "rfq_gemm.cu", "rfq_static_ws.cu"]
+SOURCES = ["rfq_api.cu", "rfq_quantize.cu", "rfq_gemm.cu", "rfq_linear_fused.cu", "rfq_static_ws.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-ftz=false", "-prec-div=true",
               "-prec-sqrt=true", "-fmad=true", "--expt-relaxed-constexpr", "-Wno-deprecated-declarations"]

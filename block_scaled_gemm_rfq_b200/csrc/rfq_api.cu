@@ -128,6 +128,25 @@ rfq_status_t gemm_impl(const void* qxc, const void* qxs, const void* qrc, const 
                                     g_encode_tiled, skip, stream));
 }
 
+rfq_status_t fused_impl(const void* x, int64_t M, int64_t K, const void* qwc, const void* qws, int64_t N, void* y,
+                        rfq_out_t y_type, int use_residual, cudaStream_t stream) {
+  if (M < 0 || N < 0 || K < 0) return RFQ_ERR_INVALID_ARG;
+  if (y_type != RFQ_OUT_F32 && y_type != RFQ_OUT_BF16) return RFQ_ERR_INVALID_ARG;
+  if (!shape_ok(M, K) || !shape_ok(N, K) || (N % 8) != 0 || M > RFQ_FUSED_MAX_M) return RFQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return RFQ_OK;
+  if (!y) return RFQ_ERR_INVALID_ARG;
+  if (!aligned16(y)) return RFQ_ERR_MISALIGNED;
+  int sms = 0;
+  rfq_status_t st = current_device(&sms);
+  if (st != RFQ_OK) return st;
+  const size_t y_bytes = static_cast<size_t>(M) * static_cast<size_t>(N) * (y_type == RFQ_OUT_BF16 ? 2u : 4u);
+  if (K == 0) return from_cuda(cudaMemsetAsync(y, 0, y_bytes, stream));
+  if (!x || !qwc || !qws) return RFQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(qwc) || !aligned16(qws)) return RFQ_ERR_MISALIGNED;
+  return from_cuda(rfq::launch_linear_fused(x, M, K, qwc, qws, N, y, y_type == RFQ_OUT_BF16, use_residual != 0, sms,
+                                            g_encode_tiled, stream));
+}
+
 }  // namespace
 
 extern "C" {
@@ -191,6 +210,7 @@ rfq_status_t rfq_linear(const void* x_bf16, int64_t M, int64_t K, const void* qw
   if (K > 0 && (workspace == nullptr || workspace_bytes < need)) return RFQ_ERR_WORKSPACE;
   if (K > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return RFQ_ERR_MISALIGNED;
   if (K > 0 && (!x_bf16 || !qw_codes || !qw_scales)) return RFQ_ERR_INVALID_ARG;
+  if (M <= RFQ_FUSED_MAX_M) return fused_impl(x_bf16, M, K, qw_codes, qw_scales, N, y, y_type, use_residual, stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t cb = align256(rfq_codes_bytes(M, K));
   const size_t sb = align256(rfq_scales_bytes(M, K));
@@ -203,13 +223,21 @@ rfq_status_t rfq_linear(const void* x_bf16, int64_t M, int64_t K, const void* qw
   return gemm_impl(qxc, qxs, qrc, qrs, qw_codes, qw_scales, M, N, K, y, y_type, stream);
 }
 
+rfq_status_t rfq_linear_fused(const void* x_bf16, int64_t M, int64_t K, const void* qw_codes, const void* qw_scales,
+                              int64_t N, void* y, rfq_out_t y_type, int use_residual, cudaStream_t stream) {
+  return fused_impl(x_bf16, M, K, qw_codes, qw_scales, N, y, y_type, use_residual, stream);
+}
+
 rfq_status_t rfq_check_device_error(cudaStream_t stream, int* detail) {
   if (detail) *detail = 0;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return RFQ_ERR_CUDA;
   unsigned int v = 0, q = 0;
   if (rfq::read_and_clear_device_error(&v) != cudaSuccess) return RFQ_ERR_CUDA;
+  unsigned int f = 0;
   if (rfq::read_and_clear_quant_error(&q) != cudaSuccess) return RFQ_ERR_CUDA;
+  if (rfq::read_and_clear_fused_error(&f) != cudaSuccess) return RFQ_ERR_CUDA;
   if (v == 0) v = q;
+  if (v == 0) v = f;
   if (detail) *detail = static_cast<int>(v);
   return v ? RFQ_ERR_TIMEOUT : RFQ_OK;
 }
@@ -218,6 +246,12 @@ rfq_status_t rfq_check_device_error(cudaStream_t stream, int* detail) {
 // its fill number `fill_index` (so a bounded wait runs out); -1 clears it.
 rfq_status_t rfq_debug_skip_next_fill(int fill_index) {
   g_skip_fill.store(fill_index < 0 ? -1 : fill_index);
+  return RFQ_OK;
+}
+
+rfq_status_t rfq_debug_fused_split(int split) {
+  if (split < 0 || split > 8) return RFQ_ERR_INVALID_ARG;
+  rfq::set_fused_split_override(split);
   return RFQ_OK;
 }
 

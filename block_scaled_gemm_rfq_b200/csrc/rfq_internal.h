@@ -21,8 +21,15 @@ cudaError_t launch_gemm(const void* qx_codes, const void* qx_scales, const void*
                         const void* qw_codes, const void* qw_scales, int64_t M, int64_t N, int64_t K, void* y,
                         bool y_bf16, int num_sms, void* encode_tiled, int skip_fill, cudaStream_t stream);
 
+// Single-kernel RFQ linear layer for M <= 64 (quantizer inside the GEMM).
+cudaError_t launch_linear_fused(const void* x, int64_t M, int64_t K, const void* qw_codes, const void* qw_scales,
+                                int64_t N, void* y, bool y_bf16, bool residual, int num_sms, void* encode_tiled,
+                                cudaStream_t stream);
+void set_fused_split_override(int split);   // 0 = automatic
+
 // Read and clear the device error words (GEMM and quantizer) of the current device.
 cudaError_t read_and_clear_device_error(unsigned int* value);
 cudaError_t read_and_clear_quant_error(unsigned int* value);
+cudaError_t read_and_clear_fused_error(unsigned int* value);
 
 }  // namespace rfq

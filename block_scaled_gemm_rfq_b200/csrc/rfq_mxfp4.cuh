@@ -1,0 +1,172 @@
+// rfq_mxfp4.cuh -- per-block MXFP4 / RFQ arithmetic shared by the stand-alone
+// quantizer (rfq_quantize.cu) and the fused quantize-and-multiply kernel
+// (rfq_linear_fused.cu).
+//
+// "Activation Outliers Matter: Robust Recovery for Quantized Multimodal LLMs",
+// section 1 (RFQ contribution paragraph): a 32-element block of X gets an E8M0
+// scale and E2M1 codes (OCP MX v1.0, section 6.3: scale exponent
+// floor(log2 amax) - emax_elem, emax_elem = 2 for E2M1; elements X / scale rounded
+// to nearest even, saturating to +-6); the residual R = X - DQ(Q(X)) is formed
+// exactly in fp32 and quantized by the same rule.
+#pragma once
+
+#include <cstdint>
+
+namespace rfq {
+
+// ---------------------------------------------------------------- arithmetic helpers
+__device__ __forceinline__ void mul2(float& o0, float& o1, float i0, float i1, float s) {
+  asm("{\n\t.reg .b64 p, q, r;\n\t"
+      "mov.b64 p, {%2, %3};\n\t"
+      "mov.b64 q, {%4, %4};\n\t"
+      "mul.rn.f32x2 r, p, q;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(o0), "=f"(o1)
+      : "f"(i0), "f"(i1), "f"(s));
+}
+
+// (o0, o1) = (a0, a1) * s + (c0, c1), each rounded once.
+__device__ __forceinline__ void fma2(float& o0, float& o1, float a0, float a1, float s, float c0, float c1) {
+  asm("{\n\t.reg .b64 p, q, c, r;\n\t"
+      "mov.b64 p, {%2, %3};\n\t"
+      "mov.b64 q, {%4, %4};\n\t"
+      "mov.b64 c, {%5, %6};\n\t"
+      "fma.rn.f32x2 r, p, q, c;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(o0), "=f"(o1)
+      : "f"(a0), "f"(a1), "f"(s), "f"(c0), "f"(c1));
+}
+
+// 8 fp32 values -> 8 E2M1 codes in one word (element i in bits 4i+3..4i), round
+// to nearest even, saturating to +-6.
+__device__ __forceinline__ uint32_t encode8(const float* v) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return out;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// bf16 pair word -> the two fp32 values (element 2j from the low half; exact).
+__device__ __forceinline__ void unpack_bf16x2(uint32_t w, float& lo, float& hi) {
+  lo = __uint_as_float(w << 16);
+  hi = __uint_as_float(w & 0xffff0000u);
+}
+
+// One word of 8 E2M1 codes -> their exact values as fp32.  The magnitudes
+// {0, .5, 1, 1.5, 2, 3, 4, 6} are bf16 0x0000, 0x3F00, 0x3F80, 0x3FC0, 0x4000,
+// 0x4040, 0x4080, 0x40C0: two 8-entry byte tables (high and low bytes) indexed by
+// the 3 magnitude bits of 4 codes at a time through byte permutes, then
+// interleaved into bf16 pairs.  The sign of a code is the sign of the element it
+// was encoded from, so it is copied from the input pair `xw[j]` (bf16 sign bits
+// 15 and 31) instead of being decoded.
+__device__ __forceinline__ void decode8(uint32_t cw, const uint32_t* xw, float* v) {
+  const uint32_t mags = cw & 0x77777777u;
+  const uint32_t sel_lo = mags & 0xffffu, sel_hi = mags >> 16;
+  const uint32_t hi0 = prmt(0x3F3F3F00u, 0x40404040u, sel_lo), lo0 = prmt(0xC0800000u, 0xC0804000u, sel_lo);
+  const uint32_t hi1 = prmt(0x3F3F3F00u, 0x40404040u, sel_hi), lo1 = prmt(0xC0800000u, 0xC0804000u, sel_hi);
+  const uint32_t pr[4] = {prmt(lo0, hi0, 0x5140u), prmt(lo0, hi0, 0x7362u), prmt(lo1, hi1, 0x5140u),
+                          prmt(lo1, hi1, 0x7362u)};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t bf2 = pr[j] | (xw[j] & 0x80008000u);
+    unpack_bf16x2(bf2, v[2 * j], v[2 * j + 1]);
+  }
+}
+
+// Per half: max(|a|, |b|) (with the XOR of the signs as sign, cleared by the
+// caller), NaN-propagating.
+__device__ __forceinline__ uint32_t bmax2_abs(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// E8M0 byte from a biased exponent field: max(bexp - 2, 0) = clamp(floor(log2 amax)
+// - 2, -127, 127) + 127; 0xFF (NaN) for a NaN/infinite amax.
+__device__ __forceinline__ uint32_t scale_byte(uint32_t bexp) {
+  return bexp == 0xFFu ? 0xFFu : (bexp >= 2u ? bexp - 2u : 0u);
+}
+
+// 2^(127 - s) and 2^(s - 127) as fp32 for a scale byte s in [0, 254].
+__device__ __forceinline__ float inv_scale(uint32_t s) { return __uint_as_float((254u - s) << 23); }
+__device__ __forceinline__ float scale_value(uint32_t s) {
+  return s == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(s << 23);
+}
+
+// Quantize one 32-element bf16 block (16 words, element 2i in the low half of
+// word i).  Outputs the E2M1 codes of Q(X) (4 words, element i in bits
+// 4(i%8)+3..4(i%8) of word i/8) and its E8M0 byte, and, with kResidual, the codes
+// and byte of Q(R), R = X - DQ(Q(X)).  A non-finite block gets scale byte 0xFF
+// for both terms (its codes are unspecified).
+template <bool kResidual>
+__device__ __forceinline__ void quantize_block(const uint32_t (&w)[16], uint32_t (&cx)[4], uint32_t& sx_out,
+                                               uint32_t (&cr)[4], uint32_t& sr_out) {
+  // ---- Q(X): block amax on bf16 magnitudes (NaN-propagating), E8M0 byte
+  uint32_t m[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = bmax2_abs(w[2 * k], w[2 * k + 1]);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) m[k] = bmax2_abs(m[k], m[k + 4]);
+  m[0] = bmax2_abs(bmax2_abs(m[0], m[2]), bmax2_abs(m[1], m[3])) & 0x7fff7fffu;
+  const uint32_t amax = max(m[0] & 0xffffu, m[0] >> 16);
+  const uint32_t sx = scale_byte(amax >> 7);
+  const uint32_t sx_eff = sx == 0xFFu ? 127u : sx;   // codes of a non-finite block are unspecified
+  const float inv_x = inv_scale(sx_eff);
+  const float neg_sc = -scale_value(sx_eff);
+
+  // Per group of 8 elements: unpack bf16 -> fp32, scale (exact), encode; then
+  // decode and form the residual R = X - DQ(Q(X)) in fp32 (exact).
+  float r[32];
+  float ra = 0.0f, rb = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float xv[8], v[8];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      unpack_bf16x2(w[4 * k + h], xv[2 * h], xv[2 * h + 1]);
+      mul2(v[2 * h], v[2 * h + 1], xv[2 * h], xv[2 * h + 1], inv_x);
+    }
+    cx[k] = encode8(v);
+    if constexpr (kResidual) {
+      float dq[8];
+      decode8(cx[k], w + 4 * k, dq);
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const int e = 8 * k + 2 * h;
+        fma2(r[e], r[e + 1], dq[2 * h], dq[2 * h + 1], neg_sc, xv[2 * h], xv[2 * h + 1]);
+        ra = fmaxf(ra, fabsf(r[e]));
+        rb = fmaxf(rb, fabsf(r[e + 1]));
+      }
+    }
+  }
+  sx_out = sx;
+
+  if constexpr (kResidual) {
+    // ---- Q(R) by the same rule
+    uint32_t sr = scale_byte(__float_as_uint(fmaxf(ra, rb)) >> 23);
+    if (sx == 0xFFu) sr = 0xFFu;
+    const float inv_r = inv_scale(sr == 0xFFu ? 127u : sr);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float v[8];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) mul2(v[2 * h], v[2 * h + 1], r[8 * k + 2 * h], r[8 * k + 2 * h + 1], inv_r);
+      cr[k] = encode8(v);
+    }
+    sr_out = sr;
+  }
+}
+
+}  // namespace rfq

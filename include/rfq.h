@@ -138,6 +138,8 @@ size_t rfq_linear_workspace_bytes(int64_t M, int64_t K, int use_residual);
  * rfq_linear -- the RFQ linear layer: rfq_quantize_mxfp4 of X into the caller's
  * workspace, then rfq_gemm against the pre-quantized weight, on one stream
  * ("requires no architectural modifications": a drop-in for the layer's GEMM).
+ * For 1 <= M <= RFQ_FUSED_MAX_M it runs rfq_linear_fused instead (same
+ * arguments checked; the workspace is then left untouched).
  *
  *   x_bf16          [M][K] bf16
  *   qw_codes/scales the weight as written by rfq_quantize_weight for [N][K]
@@ -152,6 +154,30 @@ rfq_status_t rfq_linear(const void* x_bf16, int64_t M, int64_t K,
                         void* y, rfq_out_t y_type, int use_residual,
                         void* workspace, size_t workspace_bytes,
                         cudaStream_t stream);
+
+/* Largest M that rfq_linear_fused accepts; rfq_linear uses it for 1 <= M <= this. */
+#define RFQ_FUSED_MAX_M 64
+
+/*
+ * rfq_linear_fused -- the RFQ linear layer in one kernel for short batches
+ * (M <= RFQ_FUSED_MAX_M): the quantizer runs inside the GEMM kernel, so Q(X)
+ * and Q(R) exist only in shared memory ("requantize the activation residual
+ * during GEMM", section 1).  Same codes, scales and accumulation as rfq_linear;
+ * K is split across a cluster of CTAs per 128 columns of Y and the partial
+ * sums are added in a fixed order, so Y differs from rfq_linear's only by fp32
+ * summation order.  Needs no workspace.
+ *
+ *   x_bf16          [M][K] bf16, 16-byte aligned
+ *   qw_codes/scales the weight as written by rfq_quantize_weight for [N][K]
+ *   y               [M][N] in y_type, 16-byte aligned
+ * K multiple of 32; N multiple of 8; M > RFQ_FUSED_MAX_M is
+ * RFQ_ERR_UNSUPPORTED_SHAPE.  M == 0 or N == 0 launches nothing; K == 0 writes
+ * zeros.
+ */
+rfq_status_t rfq_linear_fused(const void* x_bf16, int64_t M, int64_t K,
+                              const void* qw_codes, const void* qw_scales, int64_t N,
+                              void* y, rfq_out_t y_type, int use_residual,
+                              cudaStream_t stream);
 
 /*
  * Size of the fixed scratch array used by rfq_linear_static_workspace: 32 MiB of
@@ -196,7 +222,9 @@ rfq_status_t rfq_linear_static_workspace(const void* x_bf16, int64_t M, int64_t 
  * or RFQ_ERR_CUDA (the synchronization itself failed).  When detail is non-NULL
  * it receives the raw word (0 = none; 1..5 a wait inside rfq_gemm: 1 stage
  * load, 2 free stage, 3 accumulator ready, 4 accumulator free, 5 teardown;
- * 6 a wait of the quantizer for its TMA load).
+ * 6 a wait of the quantizer for its TMA load; the same codes 1, 2, 3, 5 for
+ * the corresponding waits of rfq_linear_fused, and 7 its quantizer warps
+ * waiting for a staged tile of X).
  */
 rfq_status_t rfq_check_device_error(cudaStream_t stream, int* detail);
 
@@ -210,6 +238,13 @@ rfq_status_t rfq_check_device_error(cudaStream_t stream, int* detail);
  * pending request.  Always returns RFQ_OK.
  */
 rfq_status_t rfq_debug_skip_next_fill(int fill_index);
+
+/*
+ * Tuning hook: make rfq_linear_fused split K over `split` CTAs (1..8, capped at
+ * the number of 256-element k-tiles) instead of choosing from the device's
+ * occupancy; 0 restores the automatic choice.  Process-wide.
+ */
+rfq_status_t rfq_debug_fused_split(int split);
 
 #ifdef __cplusplus
 }

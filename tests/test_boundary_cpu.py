@@ -76,6 +76,13 @@ def test_argument_errors_return_before_launch(lib):
     # workspace too small / missing
     assert lib.rfq_linear(_vp(A), 16, 64, _vp(A), _vp(A), 16, _vp(A), 0, 1, None, 0, None) == 7
     assert lib.rfq_linear(_vp(A), 16, 64, _vp(A), _vp(A), 16, _vp(A), 0, 1, _vp(A), 10, None) == 7
+    # fused layer: more rows than it takes, N not a multiple of 8, bad output type, bad split
+    assert lib.rfq_linear_fused(_vp(A), 65, 64, _vp(A), _vp(A), 16, _vp(A), 0, 1, None) == 2
+    assert lib.rfq_linear_fused(_vp(A), 16, 64, _vp(A), _vp(A), 12, _vp(A), 0, 1, None) == 2
+    assert lib.rfq_linear_fused(_vp(A), 16, 64, _vp(A), _vp(A), 16, _vp(A), 9, 1, None) == 1
+    assert lib.rfq_debug_fused_split(9) == 1 and lib.rfq_debug_fused_split(-1) == 1
+    assert lib.rfq_debug_fused_split(0) == 0
+    assert lib.rfq_linear_fused(None, 0, 64, None, None, 16, None, 0, 1, None) == 0
     # empty problems are valid no-ops (no device needed)
     assert lib.rfq_quantize_mxfp4(None, 0, 64, None, None, None, None, None) == 0
     assert lib.rfq_gemm(None, None, None, None, None, None, 0, 16, 64, None, 0, None) == 0
