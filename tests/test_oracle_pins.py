@@ -162,8 +162,36 @@ def test_residual_is_full_error_and_requantized_by_same_rule(oracle):
     codes_r, scales_r = oracle.quantize_f64(R)
     np.testing.assert_array_equal(codes_r, q["codes_r"])
     np.testing.assert_array_equal(scales_r, q["scales_r"])
-    # R is exactly representable in fp32 (the GPU keeps it in fp32)
+    # R is exactly representable in fp32 (and in bf16: test_residual_is_exact_in_bf16)
     np.testing.assert_array_equal(R.astype(np.float32).astype(np.float64), R)
+
+
+def test_residual_is_exact_in_bf16(oracle):
+    """|r| <= |x| elementwise (0 is a grid point) and r is a multiple of x's bf16 ulp
+    (DQ is a multiple of 2^(e-1), e >= e_x - 2), so R = X - DQ(Q(X)) is itself a bf16
+    value: computing it with one bf16 FMA involves no rounding."""
+    for seed in (14, 15):
+        bits = _rand_heavy(128, 1024, seed)
+        X = wl.bf16_bits_to_f32(bits).astype(np.float64)
+        q = oracle.quantize_bf16(bits)
+        R = X - oracle.dequantize(q["codes_x"], q["scales_x"])
+        assert np.all(np.abs(R) <= np.abs(X))
+        r32 = R.astype(np.float32)
+        np.testing.assert_array_equal(r32.astype(np.float64), R)
+        assert np.all((r32.view(np.uint32) & 0xFFFF) == 0), "a residual needs more than bf16 precision"
+    # every bf16 magnitude in [2^-8, 8) against scale 2^0 (block amax fixed at 7.5 -> e = 0)
+    mags = np.arange(0x3B80, 0x4100, dtype=np.uint16)            # 2^-8 .. just below 8
+    mags = mags[(mags & 0x7F80) != 0x7F80]
+    n = (len(mags) + 30) // 31 * 31
+    blk = np.full(n, mags[0], np.uint16)
+    blk[: len(mags)] = mags
+    blk = blk.reshape(-1, 31)
+    rows = np.concatenate([blk, np.full((blk.shape[0], 1), 0x40F0, np.uint16)], axis=1)  # 7.5 sets e = 0
+    q = oracle.quantize_bf16(rows)
+    assert np.all(q["scales_x"] == 127)
+    X = wl.bf16_bits_to_f32(rows).astype(np.float64)
+    R = X - oracle.dequantize(q["codes_x"], q["scales_x"])
+    assert np.all((R.astype(np.float32).view(np.uint32) & 0xFFFF) == 0)
 
 
 def test_residual_never_increases_error(oracle):
