@@ -20,7 +20,8 @@ __all__ = [
     "RFQError", "load_library", "library_path", "codes_bytes", "scales_bytes", "linear_workspace_bytes",
     "quantize_mxfp4", "quantize_weight", "gemm", "linear", "linear_static_workspace", "check_device_error",
     "debug_skip_next_fill", "STATIC_WORKSPACE_BYTES", "linear_fused", "linear_fused_alloc", "debug_fused_split",
-    "FUSED_MAX_M",
+    "FUSED_MAX_M", "quantize_mxfp4_t", "gemm_yt", "linear_dgrad", "linear_wgrad", "linear_wgrad_workspace_bytes",
+    "quantize_mxfp4_t_alloc", "linear_wgrad_alloc", "linear_dgrad_alloc",
     "QuantizedTensor", "quantize_mxfp4_alloc", "quantize_weight_alloc", "gemm_alloc", "linear_alloc",
     "EXPORTED_SYMBOLS", "OUT_F32", "OUT_BF16",
 ]
@@ -40,7 +41,8 @@ STATUS = {0: "RFQ_OK", 1: "RFQ_ERR_INVALID_ARG", 2: "RFQ_ERR_UNSUPPORTED_SHAPE",
 EXPORTED_SYMBOLS = (
     "rfq_status_string", "rfq_codes_bytes", "rfq_scales_bytes", "rfq_quantize_mxfp4", "rfq_quantize_weight",
     "rfq_gemm", "rfq_linear_workspace_bytes", "rfq_linear", "rfq_check_device_error", "rfq_debug_skip_next_fill",
-    "rfq_linear_static_workspace", "rfq_linear_fused", "rfq_debug_fused_split",
+    "rfq_linear_static_workspace", "rfq_linear_fused", "rfq_debug_fused_split", "rfq_quantize_mxfp4_t",
+    "rfq_gemm_yt", "rfq_linear_dgrad", "rfq_linear_wgrad_workspace_bytes", "rfq_linear_wgrad",
 )
 
 # Size of the library's fixed scratch array (RFQ_STATIC_WORKSPACE_BYTES in include/rfq.h).
@@ -84,6 +86,11 @@ def load_library():
                 "rfq_linear_static_workspace": (I, [P, I64, I64, P, P, I64, P, I, I, P]),
                 "rfq_linear_fused": (I, [P, I64, I64, P, P, I64, P, I, I, P]),
                 "rfq_debug_fused_split": (I, [I]),
+                "rfq_quantize_mxfp4_t": (I, [P, I64, I64, P, P, P, P, P]),
+                "rfq_gemm_yt": (I, [P, P, P, P, P, P, I64, I64, I64, P, I, P]),
+                "rfq_linear_dgrad": (I, [P, I64, I64, P, P, I64, P, I, I, P, SZ, P]),
+                "rfq_linear_wgrad_workspace_bytes": (SZ, [I64, I64, I64, I]),
+                "rfq_linear_wgrad": (I, [P, P, I64, I64, I64, P, I, I, P, SZ, P]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(lib, name)
@@ -182,6 +189,46 @@ def debug_fused_split(split: int):
     _check(load_library().rfq_debug_fused_split(int(split)), "rfq_debug_fused_split")
 
 
+def quantize_mxfp4_t(x, qt_codes, qt_scales, qr_codes=None, qr_scales=None, stream=None):
+    """rfq_quantize_mxfp4_t: the MXFP4 operand of x^T (x is [R][C]; blocks along R)."""
+    R, C = x.shape
+    _check(load_library().rfq_quantize_mxfp4_t(_ptr(x), R, C, _ptr(qt_codes), _ptr(qt_scales), _ptr(qr_codes),
+                                               _ptr(qr_scales), _stream(stream)), "rfq_quantize_mxfp4_t")
+
+
+def gemm_yt(qx_codes, qx_scales, qr_codes, qr_scales, qw_codes, qw_scales, M, N, K, yt, stream=None):
+    """rfq_gemm_yt: rfq_gemm writing Y^T ([N][M])."""
+    import torch
+    y_type = OUT_BF16 if yt.dtype == torch.bfloat16 else OUT_F32
+    _check(load_library().rfq_gemm_yt(_ptr(qx_codes), _ptr(qx_scales), _ptr(qr_codes), _ptr(qr_scales),
+                                      _ptr(qw_codes), _ptr(qw_scales), M, N, K, _ptr(yt), y_type, _stream(stream)),
+           "rfq_gemm_yt")
+
+
+def linear_dgrad(dy, qwt_codes, qwt_scales, K, dx, workspace, use_residual=True, stream=None):
+    """rfq_linear_dgrad: dX = dY . W (W^T pre-quantized along N by quantize_mxfp4_t)."""
+    import torch
+    M, N = dy.shape
+    y_type = OUT_BF16 if dx.dtype == torch.bfloat16 else OUT_F32
+    _check(load_library().rfq_linear_dgrad(_ptr(dy), M, N, _ptr(qwt_codes), _ptr(qwt_scales), K, _ptr(dx), y_type,
+                                           int(bool(use_residual)), _ptr(workspace), workspace.numel(),
+                                           _stream(stream)), "rfq_linear_dgrad")
+
+
+def linear_wgrad_workspace_bytes(M: int, K: int, N: int, use_residual: bool = True) -> int:
+    return int(load_library().rfq_linear_wgrad_workspace_bytes(M, K, N, int(bool(use_residual))))
+
+
+def linear_wgrad(x, dy, dw, workspace, use_residual=True, stream=None):
+    """rfq_linear_wgrad: dW [N][K] = dY^T . X with both quantized along the M tokens."""
+    import torch
+    M, K = x.shape
+    N = dy.shape[1]
+    y_type = OUT_BF16 if dw.dtype == torch.bfloat16 else OUT_F32
+    _check(load_library().rfq_linear_wgrad(_ptr(x), _ptr(dy), M, K, N, _ptr(dw), y_type, int(bool(use_residual)),
+                                           _ptr(workspace), workspace.numel(), _stream(stream)), "rfq_linear_wgrad")
+
+
 def check_device_error(stream=None):
     """Synchronize and report a bounded-wait timeout inside a kernel (raises RFQError)."""
     detail = ctypes.c_int(0)
@@ -249,6 +296,35 @@ def linear_fused_alloc(x, qw: QuantizedTensor, out_dtype=None, use_residual=True
     y = torch.empty((x.shape[0], qw.rows), dtype=out_dtype, device=x.device)
     linear_fused(x, qw.codes, qw.scales, qw.rows, y, use_residual, stream)
     return y
+
+
+def quantize_mxfp4_t_alloc(x, residual=True, stream=None) -> QuantizedTensor:
+    """The operand of x^T: rows = x's columns, K = x's rows."""
+    R, C = x.shape
+    cb, sb = codes_bytes(C, R), scales_bytes(C, R)
+    q = QuantizedTensor(C, R, _empty_u8(cb, x.device), _empty_u8(sb, x.device),
+                        _empty_u8(cb, x.device) if residual else None, _empty_u8(sb, x.device) if residual else None)
+    quantize_mxfp4_t(x, q.codes, q.scales, q.r_codes, q.r_scales, stream)
+    return q
+
+
+def linear_dgrad_alloc(dy, qwt: QuantizedTensor, out_dtype=None, use_residual=True, stream=None):
+    import torch
+    M, N = dy.shape
+    dx = torch.empty((M, qwt.rows), dtype=out_dtype or torch.bfloat16, device=dy.device)
+    ws = _empty_u8(linear_workspace_bytes(M, N, use_residual), dy.device)
+    linear_dgrad(dy, qwt.codes, qwt.scales, qwt.rows, dx, ws, use_residual, stream)
+    return dx
+
+
+def linear_wgrad_alloc(x, dy, out_dtype=None, use_residual=True, stream=None):
+    import torch
+    M, K = x.shape
+    N = dy.shape[1]
+    dw = torch.empty((N, K), dtype=out_dtype or torch.bfloat16, device=x.device)
+    ws = _empty_u8(linear_wgrad_workspace_bytes(M, K, N, use_residual), x.device)
+    linear_wgrad(x, dy, dw, ws, use_residual, stream)
+    return dw
 
 
 def linear_alloc(x, qw: QuantizedTensor, out_dtype=None, use_residual=True, stream=None):

@@ -106,7 +106,7 @@ rfq_status_t quantize_impl(const void* x, int64_t M, int64_t K, void* qc, void* 
 
 rfq_status_t gemm_impl(const void* qxc, const void* qxs, const void* qrc, const void* qrs, const void* qwc,
                        const void* qws, int64_t M, int64_t N, int64_t K, void* y, rfq_out_t y_type,
-                       cudaStream_t stream) {
+                       cudaStream_t stream, bool y_transposed = false) {
   if (M < 0 || N < 0 || K < 0) return RFQ_ERR_INVALID_ARG;
   if (y_type != RFQ_OUT_F32 && y_type != RFQ_OUT_BF16) return RFQ_ERR_INVALID_ARG;
   if ((qrc == nullptr) != (qrs == nullptr)) return RFQ_ERR_INVALID_ARG;
@@ -124,8 +124,23 @@ rfq_status_t gemm_impl(const void* qxc, const void* qxs, const void* qrc, const 
       (qrc && (!aligned16(qrc) || !aligned16(qrs))))
     return RFQ_ERR_MISALIGNED;
   const int skip = g_skip_fill.exchange(-1);
-  return from_cuda(rfq::launch_gemm(qxc, qxs, qrc, qrs, qwc, qws, M, N, K, y, y_type == RFQ_OUT_BF16, sms,
-                                    g_encode_tiled, skip, stream));
+  return from_cuda(rfq::launch_gemm(qxc, qxs, qrc, qrs, qwc, qws, M, N, K, y, y_type == RFQ_OUT_BF16,
+                                    y_transposed, sms, g_encode_tiled, skip, stream));
+}
+
+rfq_status_t quantize_t_impl(const void* x, int64_t R, int64_t C, void* qc, void* qs, void* rc, void* rs,
+                             cudaStream_t stream) {
+  if (R < 0 || C < 0) return RFQ_ERR_INVALID_ARG;
+  if (!shape_ok(C, R) || (C % 8) != 0) return RFQ_ERR_UNSUPPORTED_SHAPE;
+  if ((rc == nullptr) != (rs == nullptr)) return RFQ_ERR_INVALID_ARG;
+  if (R == 0 || C == 0) return RFQ_OK;
+  if (!x || !qc || !qs) return RFQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(qc) || !aligned16(qs) || (rc && (!aligned16(rc) || !aligned16(rs))))
+    return RFQ_ERR_MISALIGNED;
+  int sms = 0;
+  rfq_status_t st = current_device(&sms);
+  if (st != RFQ_OK) return st;
+  return from_cuda(rfq::launch_quantize_t(x, R, C, qc, qs, rc, rs, sms, g_encode_tiled, stream));
 }
 
 rfq_status_t fused_impl(const void* x, int64_t M, int64_t K, const void* qwc, const void* qws, int64_t N, void* y,
@@ -226,6 +241,59 @@ rfq_status_t rfq_linear(const void* x_bf16, int64_t M, int64_t K, const void* qw
 rfq_status_t rfq_linear_fused(const void* x_bf16, int64_t M, int64_t K, const void* qw_codes, const void* qw_scales,
                               int64_t N, void* y, rfq_out_t y_type, int use_residual, cudaStream_t stream) {
   return fused_impl(x_bf16, M, K, qw_codes, qw_scales, N, y, y_type, use_residual, stream);
+}
+
+rfq_status_t rfq_quantize_mxfp4_t(const void* x_bf16, int64_t R, int64_t C, void* qt_codes, void* qt_scales,
+                                  void* qr_codes, void* qr_scales, cudaStream_t stream) {
+  return quantize_t_impl(x_bf16, R, C, qt_codes, qt_scales, qr_codes, qr_scales, stream);
+}
+
+rfq_status_t rfq_gemm_yt(const void* qx_codes, const void* qx_scales, const void* qr_codes, const void* qr_scales,
+                         const void* qw_codes, const void* qw_scales, int64_t M, int64_t N, int64_t K, void* yt,
+                         rfq_out_t y_type, cudaStream_t stream) {
+  return gemm_impl(qx_codes, qx_scales, qr_codes, qr_scales, qw_codes, qw_scales, M, N, K, yt, y_type, stream, true);
+}
+
+rfq_status_t rfq_linear_dgrad(const void* dy_bf16, int64_t M, int64_t N, const void* qwt_codes,
+                              const void* qwt_scales, int64_t K, void* dx, rfq_out_t dx_type, int use_residual,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return rfq_linear(dy_bf16, M, N, qwt_codes, qwt_scales, K, dx, dx_type, use_residual, workspace, workspace_bytes,
+                    stream);
+}
+
+size_t rfq_linear_wgrad_workspace_bytes(int64_t M, int64_t K, int64_t N, int use_residual) {
+  if (!shape_ok(K, M) || !shape_ok(N, M)) return 0;
+  const size_t xt = align256(rfq_codes_bytes(K, M)) + align256(rfq_scales_bytes(K, M));
+  const size_t dyt = align256(rfq_codes_bytes(N, M)) + align256(rfq_scales_bytes(N, M));
+  return (use_residual ? 2 * xt : xt) + dyt;
+}
+
+rfq_status_t rfq_linear_wgrad(const void* x_bf16, const void* dy_bf16, int64_t M, int64_t K, int64_t N, void* dw,
+                              rfq_out_t dw_type, int use_residual, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
+  if (M < 0 || N < 0 || K < 0) return RFQ_ERR_INVALID_ARG;
+  if (dw_type != RFQ_OUT_F32 && dw_type != RFQ_OUT_BF16) return RFQ_ERR_INVALID_ARG;
+  if (!shape_ok(K, M) || !shape_ok(N, M) || (K % 32) != 0 || (N % 8) != 0) return RFQ_ERR_UNSUPPORTED_SHAPE;
+  if (N == 0 || K == 0) return RFQ_OK;
+  if (M == 0) return gemm_impl(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, K, N, 0, dw, dw_type, stream,
+                               true);
+  const size_t need = rfq_linear_wgrad_workspace_bytes(M, K, N, use_residual);
+  if (workspace == nullptr || workspace_bytes < need) return RFQ_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return RFQ_ERR_MISALIGNED;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t xcb = align256(rfq_codes_bytes(K, M)), xsb = align256(rfq_scales_bytes(K, M));
+  const size_t ycb = align256(rfq_codes_bytes(N, M));
+  void* qxc = ws;
+  void* qxs = ws + xcb;
+  void* qrc = use_residual ? ws + xcb + xsb : nullptr;
+  void* qrs = use_residual ? ws + 2 * xcb + xsb : nullptr;
+  uint8_t* yt = ws + (use_residual ? 2 * (xcb + xsb) : xcb + xsb);
+  rfq_status_t st = quantize_t_impl(x_bf16, M, K, qxc, qxs, qrc, qrs, stream);
+  if (st != RFQ_OK) return st;
+  st = quantize_t_impl(dy_bf16, M, N, yt, yt + ycb, nullptr, nullptr, stream);
+  if (st != RFQ_OK) return st;
+  // dW^T [K][N] = (X^T)^ . (dY^T)^T, written transposed: dW [N][K]
+  return gemm_impl(qxc, qxs, qrc, qrs, yt, yt + ycb, K, N, M, dw, dw_type, stream, true);
 }
 
 rfq_status_t rfq_check_device_error(cudaStream_t stream, int* detail) {

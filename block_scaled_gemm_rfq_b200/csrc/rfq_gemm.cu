@@ -132,7 +132,7 @@ __device__ __forceinline__ uint32_t mma_idesc(uint32_t sf_id) {
          | (sf_id << 29);                        // A scale-factor id
 }
 
-template <int kPair, bool kResidual, bool kBf16Out>
+template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut>
 __global__ void __launch_bounds__(kThreads, 1)
     rfq_gemm_kernel(const __grid_constant__ Maps maps, const GemmParams p) {
   using L = Layout<kPair>;
@@ -336,7 +336,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       const int row = (mb * kPair + static_cast<int>(rank)) * kBM + quad * 32 + lane;
       const int col0 = nb * kBN + half * 128;
-      if (row < p.M) {
+      if constexpr (kTransOut) {
+        // Y^T [N][M]: for each column the warp's 32 lanes hold 32 consecutive rows,
+        // so one store per column writes 32 neighbouring elements of a row of Y^T.
+        if (row < p.M) {
+#pragma unroll
+          for (int i = 0; i < 128; ++i) {
+            if (col0 + i < p.N) {
+              const float f = __uint_as_float(v[i >> 5][i & 31]);
+              const int64_t off = static_cast<int64_t>(col0 + i) * p.M + row;
+              if (kBf16Out) static_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(f);
+              else static_cast<float*>(p.y)[off] = f;
+            }
+          }
+        }
+      } else if (row < p.M) {
         if (kBf16Out) {
           __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(row) * p.N + col0;
 #pragma unroll
@@ -377,9 +391,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int kPair, bool kResidual, bool kBf16Out>
+template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut>
 cudaError_t launch_typed(const Maps& maps, const GemmParams& p, int grid, cudaStream_t stream) {
-  auto kernel = rfq_gemm_kernel<kPair, kResidual, kBf16Out>;
+  auto kernel = rfq_gemm_kernel<kPair, kResidual, kBf16Out, kTransOut>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<kPair>::kSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -401,7 +415,7 @@ cudaError_t launch_typed(const Maps& maps, const GemmParams& p, int grid, cudaSt
   return cudaGetLastError();
 }
 
-template <int kPair>
+template <int kPair, bool kTransOut>
 cudaError_t launch_mode(const Maps& maps, GemmParams p, int64_t M, bool residual, bool y_bf16, int num_sms,
                         cudaStream_t stream) {
   const int64_t num_mb = (M + kBM * kPair - 1) / (kBM * kPair);
@@ -410,17 +424,18 @@ cudaError_t launch_mode(const Maps& maps, GemmParams p, int64_t M, bool residual
   if (units > p.num_tiles) units = p.num_tiles;
   const int grid = units * kPair;
   if (residual)
-    return y_bf16 ? launch_typed<kPair, true, true>(maps, p, grid, stream)
-                  : launch_typed<kPair, true, false>(maps, p, grid, stream);
-  return y_bf16 ? launch_typed<kPair, false, true>(maps, p, grid, stream)
-                : launch_typed<kPair, false, false>(maps, p, grid, stream);
+    return y_bf16 ? launch_typed<kPair, true, true, kTransOut>(maps, p, grid, stream)
+                  : launch_typed<kPair, true, false, kTransOut>(maps, p, grid, stream);
+  return y_bf16 ? launch_typed<kPair, false, true, kTransOut>(maps, p, grid, stream)
+                : launch_typed<kPair, false, false, kTransOut>(maps, p, grid, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm(const void* qx_codes, const void* qx_scales, const void* qr_codes, const void* qr_scales,
                         const void* qw_codes, const void* qw_scales, int64_t M, int64_t N, int64_t K, void* y,
-                        bool y_bf16, int num_sms, void* encode_tiled, int skip_fill, cudaStream_t stream) {
+                        bool y_bf16, bool y_transposed, int num_sms, void* encode_tiled, int skip_fill,
+                        cudaStream_t stream) {
   EncodeTiledFn encode = reinterpret_cast<EncodeTiledFn>(encode_tiled);
   const bool residual = qr_codes != nullptr;
   // CTA pairs once there are rows for both CTAs of a pair; single CTAs for short M.
@@ -445,8 +460,11 @@ cudaError_t launch_gemm(const void* qx_codes, const void* qx_scales, const void*
   p.num_nb = static_cast<int>((N + kBN - 1) / kBN);
   p.num_tiles = 0;
   p.skip_fill = skip_fill;
-  return pair ? launch_mode<2>(maps, p, M, residual, y_bf16, num_sms, stream)
-              : launch_mode<1>(maps, p, M, residual, y_bf16, num_sms, stream);
+  if (y_transposed)
+    return pair ? launch_mode<2, true>(maps, p, M, residual, y_bf16, num_sms, stream)
+                : launch_mode<1, true>(maps, p, M, residual, y_bf16, num_sms, stream);
+  return pair ? launch_mode<2, false>(maps, p, M, residual, y_bf16, num_sms, stream)
+              : launch_mode<1, false>(maps, p, M, residual, y_bf16, num_sms, stream);
 }
 
 cudaError_t read_and_clear_device_error(unsigned int* value) {

@@ -13,13 +13,18 @@ namespace rfq {
 cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, void* qx_codes, void* qx_scales, void* qr_codes,
                             void* qr_scales, int num_sms, void* encode_tiled, cudaStream_t stream);
 
-// Kernel 2: RFQ GEMM.  qr_codes == nullptr selects the plain MXFP4 GEMM.
+// Kernel 1t: quantizer of X^T for a row-major X [R][C] (blocks along R).
+cudaError_t launch_quantize_t(const void* x, int64_t R, int64_t C, void* qt_codes, void* qt_scales, void* qr_codes,
+                              void* qr_scales, int num_sms, void* encode_tiled, cudaStream_t stream);
+
+// Kernel 2: RFQ GEMM (y_transposed: Y written as [N][M]).  qr_codes == nullptr selects the plain MXFP4 GEMM.
 // `encode_tiled` is the driver's cuTensorMapEncodeTiled.  `skip_fill` >= 0 makes
 // the producer of CTA 0 skip that stage fill (fault injection for the bounded
 // waits; -1 in normal use).
 cudaError_t launch_gemm(const void* qx_codes, const void* qx_scales, const void* qr_codes, const void* qr_scales,
                         const void* qw_codes, const void* qw_scales, int64_t M, int64_t N, int64_t K, void* y,
-                        bool y_bf16, int num_sms, void* encode_tiled, int skip_fill, cudaStream_t stream);
+                        bool y_bf16, bool y_transposed, int num_sms, void* encode_tiled, int skip_fill,
+                        cudaStream_t stream);
 
 // Single-kernel RFQ linear layer for M <= 64 (quantizer inside the GEMM).
 cudaError_t launch_linear_fused(const void* x, int64_t M, int64_t K, const void* qw_codes, const void* qw_scales,

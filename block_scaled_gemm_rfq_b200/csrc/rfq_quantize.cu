@@ -99,6 +99,30 @@ __device__ __forceinline__ void store_scale(uint8_t* scales, uint32_t s, bool va
   }
 }
 
+// Zero the padding bytes of a scale array in the MMA layout: rows [rows, rows_pad)
+// entirely, and blocks [Kb, 4 * kb4_per_tile) of the real rows.  Grid-strided over
+// all threads of the launch.
+__device__ __forceinline__ void zero_scale_padding(uint8_t* sx, uint8_t* sr, uint32_t rows, uint32_t Kb,
+                                                   uint32_t kb4_per_tile, uint32_t rows_pad, uint32_t tid,
+                                                   uint32_t nthreads) {
+  const uint32_t pad_words = (rows_pad - rows) * kb4_per_tile;
+  for (uint32_t t = tid; t < pad_words; t += nthreads) {
+    const uint32_t r = rows + t / kb4_per_tile, kb4 = t % kb4_per_tile;
+    const uint32_t off = scale_word_offset(r, kb4, kb4_per_tile);
+    *reinterpret_cast<uint32_t*>(sx + off) = 0u;
+    if (sr) *reinterpret_cast<uint32_t*>(sr + off) = 0u;
+  }
+  const uint32_t tail = kb4_per_tile * 4 - Kb;   // 0..3 pad blocks per real row
+  if (tail > 0) {
+    for (uint32_t t = tid; t < rows * tail; t += nthreads) {
+      const uint32_t r = t / tail, kb = Kb + t % tail;
+      const uint32_t off = scale_word_offset(r, kb >> 2, kb4_per_tile) + (kb & 3);
+      sx[off] = 0;
+      if (sr) sr[off] = 0;
+    }
+  }
+}
+
 // kWide: X seen as [blocks/2][128 bytes] with a 128-byte swizzle (needs an even
 // block count); otherwise as [blocks][64 bytes] with a 64-byte swizzle.  Either
 // way a lane's four 16-byte reads of its block hit distinct banks.
@@ -210,29 +234,144 @@ __global__ void __launch_bounds__(kThreads, RFQ_Q_CTAS_PER_SM)
   // ---- zero padding of the scale arrays: rows [M, rows_pad) and blocks [Kb, 4*kb4) of real rows
   // (stores to buffers the previous kernel on the stream may still read: wait for it)
   griddep_wait();
-  const uint32_t tid = blockIdx.x * kThreads + threadIdx.x;
-  const uint32_t nthreads = gridDim.x * kThreads;
-  const uint32_t pad_words = (p.rows_pad - p.M) * p.kb4_per_tile;
-  for (uint32_t t = tid; t < pad_words; t += nthreads) {
-    const uint32_t r = p.M + t / p.kb4_per_tile, kb4 = t % p.kb4_per_tile;
-    const uint32_t off = scale_word_offset(r, kb4, p.kb4_per_tile);
-    *reinterpret_cast<uint32_t*>(p.qx_scales + off) = 0u;
-    if (kResidual) *reinterpret_cast<uint32_t*>(p.qr_scales + off) = 0u;
+  zero_scale_padding(p.qx_scales, kResidual ? p.qr_scales : nullptr, p.M, p.Kb, p.kb4_per_tile, p.rows_pad,
+                     blockIdx.x * kThreads + threadIdx.x, gridDim.x * kThreads);
+}
+
+// ---------------------------------------------------------------- transposed quantizer
+// Quantizes X^T for a row-major bf16 X [R][C]: operand row c of the output is
+// column c of X, and its 32-element blocks run down 32 consecutive rows of X.
+// A warp takes units of 32 rows x 64 columns (4 KiB, one TMA box, kTStages in
+// flight); lane l reads, for each of the 32 rows, the 32-bit word holding columns
+// 2l and 2l+1 (conflict-free: a row's 32 words), regroups the halves into the
+// pair layout of a block (byte permutes) and quantizes the two columns' blocks
+// with the same per-block arithmetic as the row quantizer.  Units are ordered
+// row-block fastest, so warps running at the same time write neighbouring 16-byte
+// pieces of the same output rows.
+constexpr int kTWarps = 8;
+constexpr int kTThreads = kTWarps * 32;
+constexpr int kTStages = 3;
+constexpr uint32_t kTUnitBytes = 32 * 128;
+constexpr uint32_t kTSmemBytes = kTWarps * kTStages * kTUnitBytes + kTWarps * kTStages * 8 + 1024;
+
+struct QuantTParams {
+  uint8_t* qt_codes;
+  uint8_t* qt_scales;
+  uint8_t* qr_codes;
+  uint8_t* qr_scales;
+  uint32_t R;             // rows of X = K of the operand
+  uint32_t C;             // columns of X = rows of the operand
+  uint32_t Rb;            // R / 32: blocks per operand row
+  uint32_t kb4_per_tile;  // ceil(Rb / 4)
+  uint32_t rows_pad;      // ceil(C / 128) * 128
+  uint32_t num_ct;        // ceil(C / 64)
+  uint32_t num_units;     // Rb * num_ct
+};
+
+template <bool kResidual>
+__global__ void __launch_bounds__(kTThreads, 2)
+    rfq_quantize_t_kernel(const __grid_constant__ CUtensorMap tm_x, const QuantTParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint8_t* ring = smem + warp * (kTStages * kTUnitBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTWarps * kTStages * kTUnitBytes) + warp * kTStages;
+  volatile int abort_flag = 0;
+
+  const uint32_t gw = blockIdx.x * kTWarps + warp;
+  const uint32_t GW = gridDim.x * kTWarps;
+  const uint32_t n_my = p.num_units > gw ? (p.num_units - gw + GW - 1) / GW : 0;
+  auto issue = [&](uint32_t k, int st) {
+    const uint32_t u = gw + k * GW;
+    const uint32_t rt = u % p.Rb, ct = u / p.Rb;
+    mbar_arrive_expect_tx(&bars[st], kTUnitBytes);
+    tma_load_2d(ring + st * kTUnitBytes, &tm_x, &bars[st], static_cast<int>(ct * 64), static_cast<int>(rt * 32));
+  };
+
+  griddep_launch_dependents();
+  if (lane == 0) {
+    for (int st = 0; st < kTStages; ++st) mbar_init(&bars[st], 1);
+    fence_mbar_init();
+    griddep_wait();   // X may be written by the previous kernel on the stream
+    for (uint32_t k = 0; k < kTStages && k < n_my; ++k) issue(k, static_cast<int>(k));
   }
-  const uint32_t tail = p.kb4_per_tile * 4 - p.Kb;   // 0..3 pad blocks per real row
-  if (tail > 0) {
-    for (uint32_t t = tid; t < p.M * tail; t += nthreads) {
-      const uint32_t r = t / tail, kb = p.Kb + t % tail;
-      const uint32_t off = scale_word_offset(r, kb >> 2, p.kb4_per_tile) + (kb & 3);
-      p.qx_scales[off] = 0;
-      if (kResidual) p.qr_scales[off] = 0;
+  __syncwarp();
+
+  uint32_t i = 0;
+  for (; i < n_my; ++i) {
+    const int st = static_cast<int>(i % kTStages);
+    const bool ok = mbar_wait(&bars[st], (i / kTStages) & 1u, &abort_flag, &g_quant_error, kErrQuantWait);
+    if (!__all_sync(0xffffffffu, ok)) break;
+    uint32_t wr[32];
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(ring + st * kTUnitBytes) + lane;
+#pragma unroll
+    for (int r = 0; r < 32; ++r) wr[r] = src[r * 32];
+    __syncwarp();
+    if (lane == 0 && i + kTStages < n_my) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue(i + kTStages, st);
+    }
+    const uint32_t u = gw + i * GW;
+    const uint32_t rt = u % p.Rb, ct = u / p.Rb;
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+      // element 2j of the block = row 2j (low half), 2j+1 = row 2j+1 (high half)
+      uint32_t w[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) w[j] = prmt(wr[2 * j], wr[2 * j + 1], h ? 0x7632u : 0x5410u);
+      uint32_t cx[4], cr[4], sx, sr;
+      quantize_block<kResidual>(w, cx, sx, cr, sr);
+      const uint32_t c = ct * 64 + 2 * lane + h;
+      if (c < p.C) {
+        const size_t code_off = static_cast<size_t>(c) * (p.R / 2) + rt * 16;
+        const uint32_t sf_off = scale_word_offset(c, rt >> 2, p.kb4_per_tile) + (rt & 3);
+        *reinterpret_cast<uint4*>(p.qt_codes + code_off) = make_uint4(cx[0], cx[1], cx[2], cx[3]);
+        p.qt_scales[sf_off] = static_cast<uint8_t>(sx);
+        if constexpr (kResidual) {
+          *reinterpret_cast<uint4*>(p.qr_codes + code_off) = make_uint4(cr[0], cr[1], cr[2], cr[3]);
+          p.qr_scales[sf_off] = static_cast<uint8_t>(sr);
+        }
+      }
     }
   }
+
+  if (i < n_my && lane == 0) {
+    // A wait ran out: let this warp's outstanding copies land before leaving.
+    int never = 0;
+    for (uint32_t k = i; k < n_my && k < i + kTStages; ++k)
+      mbar_wait(&bars[k % kTStages], static_cast<uint32_t>((k / kTStages) & 1), &never, &g_quant_error,
+                kErrQuantWait);
+  }
+
+  griddep_wait();   // the padding stores may hit buffers the previous kernel still reads
+  zero_scale_padding(p.qt_scales, kResidual ? p.qr_scales : nullptr, p.C, p.Rb, p.kb4_per_tile, p.rows_pad,
+                     blockIdx.x * kTThreads + threadIdx.x, gridDim.x * kTThreads);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+template <bool kResidual>
+cudaError_t launch_t_typed(const CUtensorMap& tm, const QuantTParams& p, int grid, cudaStream_t stream) {
+  auto kernel = rfq_quantize_t_kernel<kResidual>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTSmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kTThreads);
+  cfg.dynamicSmemBytes = kTSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see griddep_wait()
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kernel, tm, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 
 #ifndef RFQ_Q_WIDE
 #define RFQ_Q_WIDE 1
@@ -305,6 +444,41 @@ cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, void* qx_codes,
   if (qr_codes)
     return word ? launch_width<true, true>(wide, tm, p, g, stream) : launch_width<true, false>(wide, tm, p, g, stream);
   return word ? launch_width<false, true>(wide, tm, p, g, stream) : launch_width<false, false>(wide, tm, p, g, stream);
+}
+
+cudaError_t launch_quantize_t(const void* x, int64_t R, int64_t C, void* qt_codes, void* qt_scales, void* qr_codes,
+                              void* qr_scales, int num_sms, void* encode_tiled, cudaStream_t stream) {
+  QuantTParams p;
+  p.qt_codes = static_cast<uint8_t*>(qt_codes);
+  p.qt_scales = static_cast<uint8_t*>(qt_scales);
+  p.qr_codes = static_cast<uint8_t*>(qr_codes);
+  p.qr_scales = static_cast<uint8_t*>(qr_scales);
+  p.R = static_cast<uint32_t>(R);
+  p.C = static_cast<uint32_t>(C);
+  p.Rb = static_cast<uint32_t>(R / 32);
+  p.kb4_per_tile = (p.Rb + 3) / 4;
+  p.rows_pad = static_cast<uint32_t>((C + 127) / 128 * 128);
+  p.num_ct = static_cast<uint32_t>((C + 63) / 64);
+  p.num_units = p.Rb * p.num_ct;
+
+  // X as [R][C] 16-bit elements; boxes of 64 columns x 32 rows, no swizzle, zeros
+  // past the last column.
+  CUtensorMap tm;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(R)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(C) * 2};
+  cuuint32_t box[2] = {64u, 32u};
+  cuuint32_t elem_strides[2] = {1, 1};
+  EncodeTiledFn encode = reinterpret_cast<EncodeTiledFn>(encode_tiled);
+  if (encode(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(x), dims, strides, box, elem_strides,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  int64_t grid = (static_cast<int64_t>(p.num_units) + kTWarps - 1) / kTWarps;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 2;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  return qr_codes ? launch_t_typed<true>(tm, p, static_cast<int>(grid), stream)
+                  : launch_t_typed<false>(tm, p, static_cast<int>(grid), stream);
 }
 
 cudaError_t read_and_clear_quant_error(unsigned int* value) {

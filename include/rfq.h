@@ -130,6 +130,34 @@ rfq_status_t rfq_gemm(const void* qx_codes, const void* qx_scales,
                       int64_t M, int64_t N, int64_t K,
                       void* y, rfq_out_t y_type, cudaStream_t stream);
 
+/*
+ * rfq_quantize_mxfp4_t -- quantize the transpose of a row-major bf16 matrix, for the
+ * backward GEMMs of a training step (whose contractions run over a different axis
+ * than the forward's; the paper frames RFQ as FP4 *training*-aware, section 1, and
+ * gives no backward rule, so gradients pass the quantizers unchanged: straight
+ * through).  X is [R][C]; the output is the operand of X^T ([C][R], 32-element
+ * blocks along R) in exactly the layouts rfq_quantize_mxfp4 writes for a [C][R]
+ * matrix: codes rfq_codes_bytes(C, R), scales rfq_scales_bytes(C, R).  Same rules
+ * (scale, rounding, residual R^T = X^T - DQ(Q(X^T)) when qr_* are given).
+ *
+ *   x_bf16   [R][C] bf16, 16-byte aligned; R a multiple of 32, C a multiple of 8
+ * R == 0 or C == 0 launches nothing.  Every byte of the scale arrays is written.
+ */
+rfq_status_t rfq_quantize_mxfp4_t(const void* x_bf16, int64_t R, int64_t C,
+                                  void* qt_codes, void* qt_scales,
+                                  void* qr_codes, void* qr_scales,
+                                  cudaStream_t stream);
+
+/*
+ * rfq_gemm_yt -- rfq_gemm writing the transposed product: yt is [N][M] with
+ * yt[n][m] = Y[m][n].  Same operands, rules and accumulation as rfq_gemm.
+ */
+rfq_status_t rfq_gemm_yt(const void* qx_codes, const void* qx_scales,
+                         const void* qr_codes, const void* qr_scales,
+                         const void* qw_codes, const void* qw_scales,
+                         int64_t M, int64_t N, int64_t K,
+                         void* yt, rfq_out_t y_type, cudaStream_t stream);
+
 /* Workspace bytes rfq_linear needs for an [M][K] activation: codes and scales
  * of Q(X) and, when use_residual, of Q(R), each sub-buffer 256-byte aligned. */
 size_t rfq_linear_workspace_bytes(int64_t M, int64_t K, int use_residual);
@@ -154,6 +182,42 @@ rfq_status_t rfq_linear(const void* x_bf16, int64_t M, int64_t K,
                         void* y, rfq_out_t y_type, int use_residual,
                         void* workspace, size_t workspace_bytes,
                         cudaStream_t stream);
+
+/*
+ * Backward GEMMs of the layer Y = X W^T (straight-through: dL/dX ~ dL/dX^, dL/dW ~
+ * dL/dW^).  The residual pathway stays on the activation-side operand of each
+ * GEMM, as in the forward (section 1: activation quantization is the dominant
+ * error; weights stay plain MXFP4).
+ *
+ * rfq_linear_dgrad -- dX [M][K] = (DQ(Q(dY)) [+ DQ(Q(R_dY))]) . DQ(Q(W^T))^T: the
+ * contraction runs over N, so W enters as W^T quantized along N
+ * (rfq_quantize_mxfp4_t of W [N][K], no residual: qwt_* with rows K, K-dimension
+ * N).  This is rfq_linear with X := dY and the weight operand := W^T; arguments
+ * and workspace (rfq_linear_workspace_bytes(M, N, use_residual)) as there.
+ */
+rfq_status_t rfq_linear_dgrad(const void* dy_bf16, int64_t M, int64_t N,
+                              const void* qwt_codes, const void* qwt_scales, int64_t K,
+                              void* dx, rfq_out_t dx_type, int use_residual,
+                              void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream);
+
+/* Workspace bytes of rfq_linear_wgrad: Q(X^T) [and Q(R^T)] [K][M] and Q(dY^T) [N][M],
+ * each sub-buffer 256-byte aligned; 0 for unsupported shapes. */
+size_t rfq_linear_wgrad_workspace_bytes(int64_t M, int64_t K, int64_t N, int use_residual);
+
+/*
+ * rfq_linear_wgrad -- dW [N][K] = sum over the M tokens of dY[m][n] . X^[m][k], with
+ * both operands quantized along M (the contraction): X^T with the residual pathway
+ * (the forward activation), dY^T plain.  Runs rfq_quantize_mxfp4_t on X and dY and
+ * rfq_gemm_yt (A = X^T, B = dY^T, so the [K][N] product is written as [N][K]).
+ *
+ *   x_bf16 [M][K], dy_bf16 [M][N], bf16, 16-byte aligned; dw [N][K] in dw_type
+ * M a multiple of 32, K a multiple of 32, N a multiple of 8.  M == 0 writes zeros.
+ */
+rfq_status_t rfq_linear_wgrad(const void* x_bf16, const void* dy_bf16, int64_t M, int64_t K, int64_t N,
+                              void* dw, rfq_out_t dw_type, int use_residual,
+                              void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream);
 
 /* Largest M that rfq_linear_fused accepts; rfq_linear uses it for 1 <= M <= this. */
 #define RFQ_FUSED_MAX_M 64

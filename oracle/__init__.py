@@ -219,3 +219,36 @@ def rfq_linear(x_bits: np.ndarray, w_bits: np.ndarray, residual: bool = True, us
         use_loops = A.shape[0] * B.shape[0] * A.shape[1] <= 64 * 1024 * 1024
     Y, absY = gemm_loops(A, B) if use_loops else gemm_blas(A, B)
     return Y, float(absY.max()) if absY.size else 0.0, absY
+
+
+# ----------------------------------------------------------------------------- backward GEMMs
+# The paper frames RFQ as aware of FP4 *training* (section 1, the RFQ paragraph:
+# "fully differentiable and training-aware") but states no backward rule.  The
+# plainest reading is the straight-through estimator: the quantizers pass the
+# gradient unchanged, and the two backward GEMMs of Y = X W^T are themselves run on
+# MXFP4 operands quantized along *their* contraction axis, with the residual
+# pathway on the activation-side operand as in the forward.
+
+
+def quantize_transposed(x_bits: np.ndarray, residual: bool = True):
+    """MXFP4 quantization of X^T for a [R, C] bf16 matrix: blocks of 32 run down the
+    rows of X (the definition: transpose, then the row rule of ``quantize_bf16``)."""
+    return quantize_bf16(np.ascontiguousarray(np.asarray(x_bits, dtype=np.uint16).T), residual=residual)
+
+
+def rfq_dgrad(dy_bits: np.ndarray, w_bits: np.ndarray, residual: bool = True, use_loops=None):
+    """dX [M, K] = (DQ(Q(dY)) + DQ(Q(R_dY))) . DQ(Q(W^T))^T: the contraction runs over N,
+    so dY [M, N] is quantized along its rows and W [N, K] along its columns.
+    Returns (dX, S, absY) as ``rfq_linear``."""
+    wt = np.ascontiguousarray(np.asarray(w_bits, dtype=np.uint16).T)
+    return rfq_linear(dy_bits, wt, residual=residual, use_loops=use_loops)
+
+
+def rfq_wgrad(x_bits: np.ndarray, dy_bits: np.ndarray, residual: bool = True, use_loops=None):
+    """dW [N, K] = sum over the M tokens of dY[m, n] (X^[m, k]), both operands quantized
+    along M; X carries the residual pathway.  Computed as the RFQ product of X^T [K, M]
+    (activation, with residual) and dY^T [N, M], transposed.  Returns (dW, S, absY^T)."""
+    xt = np.ascontiguousarray(np.asarray(x_bits, dtype=np.uint16).T)
+    dyt = np.ascontiguousarray(np.asarray(dy_bits, dtype=np.uint16).T)
+    Y, S, absY = rfq_linear(xt, dyt, residual=residual, use_loops=use_loops)
+    return np.ascontiguousarray(Y.T), S, np.ascontiguousarray(absY.T)

@@ -303,6 +303,59 @@ def test_rfq_recovers_activation_fidelity(oracle):
 
 
 # --------------------------------------------------------------------------- scale layout
+def _representable(rows, cols, seed, axis):
+    """bf16 matrix whose 32-element blocks along `axis` are exactly MXFP4: grid
+    values times a per-block power of two (block max on the grid's top codes)."""
+    rng = np.random.default_rng(seed)
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6])
+    vals = rng.choice(grid, (rows, cols)) * rng.choice([-1.0, 1.0], (rows, cols))
+    if axis == 1:
+        v = vals.reshape(rows, cols // 32, 32)
+        v[:, :, 0] = 6.0
+        v *= np.exp2(rng.integers(-20, 20, (rows, cols // 32, 1)))
+        vals = v.reshape(rows, cols)
+    else:
+        v = vals.reshape(rows // 32, 32, cols)
+        v[:, 0, :] = 6.0
+        v *= np.exp2(rng.integers(-20, 20, (rows // 32, 1, cols)))
+        vals = v.reshape(rows, cols)
+    return wl.f64_to_bf16_bits(vals), vals
+
+
+def test_transposed_quantizer_definition_and_identity(oracle):
+    """quantize_transposed(X) is the row rule on X^T; on blocks exactly
+    representable along the rows of X it dequantizes to X^T exactly, with an
+    all-zero residual."""
+    bits, vals = _representable(96, 40, 31, axis=0)
+    q = oracle.quantize_transposed(bits)
+    np.testing.assert_array_equal(oracle.dequantize(q["codes_x"], q["scales_x"]), vals.T)
+    assert not q["codes_r"].any() and not q["scales_r"].any()
+    q2 = oracle.quantize_bf16(np.ascontiguousarray(bits.T))
+    for k in q:
+        np.testing.assert_array_equal(q[k], q2[k])
+
+
+def test_backward_gemms_straight_through_closed_form(oracle):
+    """With operands exactly MXFP4 along each GEMM's contraction axis, the
+    straight-through backward GEMMs are the plain products dX = dY . W and
+    dW = dY^T . X (float64, exact inputs)."""
+    M, N, K = 64, 64, 96
+    dy_bits, dy = _representable(M, N, 41, axis=1)     # dgrad: dY along N (its rows)
+    w_bits, w = _representable(N, K, 42, axis=0)       # dgrad: W along N (its columns)
+    dX, S, _ = oracle.rfq_dgrad(dy_bits, w_bits)
+    np.testing.assert_allclose(dX, dy @ w, rtol=0, atol=1e-12 * S)
+    x_bits, x = _representable(M, K, 43, axis=0)       # wgrad: X along M (its columns)
+    dy2_bits, dy2 = _representable(M, N, 44, axis=0)   # wgrad: dY along M
+    dW, S2, _ = oracle.rfq_wgrad(x_bits, dy2_bits)
+    np.testing.assert_allclose(dW, dy2.T @ x, rtol=0, atol=1e-12 * S2)
+    # and on general inputs the wgrad residual term is the RFQ term of X^T
+    xg = _rand_heavy(64, 96, 45)
+    dW_on, _, _ = oracle.rfq_wgrad(xg, dy2_bits, residual=True)
+    dW_off, _, _ = oracle.rfq_wgrad(xg, dy2_bits, residual=False)
+    exact = dy2.T @ wl.bf16_bits_to_f32(xg).astype(np.float64)
+    assert np.linalg.norm(dW_on - exact) < np.linalg.norm(dW_off - exact)
+
+
 def test_mma_scale_layout_known_offsets_and_bijection(oracle):
     Kb = 10                                   # Kb_pad = 12 -> 3 atoms per 128-row tile
     assert oracle.mma_scale_offset(0, 0, Kb) == 0
