@@ -259,6 +259,47 @@ def time_stream(fns, reps):
     return a.elapsed_time(b) / (reps * len(fns))
 
 
+def time_training(rfq, wk, flush, fp4_peak, hbm_peak):
+    """Backward pass of the FFN layer (straight-through): the transposed quantizer on
+    X and dY, dgrad (dX = dY . W, contraction over N) and wgrad (dW = dY^T . X,
+    contraction over the M tokens), each GEMM timed alone after an L2 flush."""
+    import numpy as np
+    import torch
+    M, K, N = wk.M, wk.K, wk.N
+    x = to_device_bf16(wk.x_bits)
+    w = to_device_bf16(wk.w_bits)
+    dy = torch.randn((M, N), device="cuda", generator=torch.Generator("cuda").manual_seed(5)).mul_(1e-3)
+    dy = dy.to(torch.bfloat16)
+    out = {}
+    # transposed quantizers
+    qxt = rfq.quantize_mxfp4_t_alloc(x, residual=True)
+    t = time_kernel(lambda: rfq.quantize_mxfp4_t(x, qxt.codes, qxt.scales, qxt.r_codes, qxt.r_scales), 20, flush)
+    out["quantize_t_x"] = {"shape": [M, K], "us": 1e3 * statistics.mean(t),
+                           "gbs": quantize_bytes(M, K, True) / (statistics.mean(t) * 1e-3) / 1e9}
+    out["quantize_t_x"]["frac_hbm"] = out["quantize_t_x"]["gbs"] / hbm_peak
+    qdyt = rfq.quantize_mxfp4_t_alloc(dy, residual=False)
+    t = time_kernel(lambda: rfq.quantize_mxfp4_t(dy, qdyt.codes, qdyt.scales), 20, flush)
+    out["quantize_t_dy"] = {"shape": [M, N], "us": 1e3 * statistics.mean(t),
+                            "gbs": quantize_bytes(M, N, False) / (statistics.mean(t) * 1e-3) / 1e9}
+    # dgrad: A = Q(dY) [M][N] (+ residual), B = Q(W^T) [K][N] -> dX [M][K]
+    qdy = rfq.quantize_mxfp4_alloc(dy, residual=True)
+    qwt = rfq.quantize_mxfp4_t_alloc(w, residual=False)
+    dx = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    t = time_kernel(lambda: rfq.gemm(qdy.codes, qdy.scales, qdy.r_codes, qdy.r_scales, qwt.codes, qwt.scales,
+                                     M, K, N, dx), 10, flush)
+    f = 4.0 * M * N * K
+    out["dgrad_gemm"] = {"us": 1e3 * statistics.mean(t), "tflops_executed": f / (statistics.mean(t) * 1e-3) / 1e12}
+    out["dgrad_gemm"]["frac_fp4_peak"] = out["dgrad_gemm"]["tflops_executed"] / fp4_peak
+    # wgrad: A = Q(X^T) [K][M] (+ residual), B = Q(dY^T) [N][M] -> dW [N][K] (transposed store)
+    dw = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+    t = time_kernel(lambda: rfq.gemm_yt(qxt.codes, qxt.scales, qxt.r_codes, qxt.r_scales, qdyt.codes, qdyt.scales,
+                                        K, N, M, dw), 10, flush)
+    out["wgrad_gemm"] = {"us": 1e3 * statistics.mean(t), "tflops_executed": f / (statistics.mean(t) * 1e-3) / 1e12}
+    out["wgrad_gemm"]["frac_fp4_peak"] = out["wgrad_gemm"]["tflops_executed"] / fp4_peak
+    rfq.check_device_error()
+    return out
+
+
 def quantize_bytes(M, K, residual):
     """Algorithmic HBM bytes of the fused quantizer: read X once (2 B/elem), write codes
     (0.5 B/elem) and scales (1 B per 32 elements) per output."""
@@ -393,6 +434,7 @@ def run_cuda(args, rank, world, local):
                 row["rfq" if res else "off"] = cell
             sweep[str(Ms)] = row
         extra["m_sweep_rfq_linear"] = sweep
+        extra["training_ffn"] = time_training(rfq, wk, flush, fp4_peak, hbm_peak)
 
     # end to end through the public API with host buffers: pinned X, W in; Y out
     xh = torch.from_numpy(wk.x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()

@@ -86,6 +86,16 @@ def _load():
             lib.oracle_mma_scale_offset.argtypes = [I64, I64, I64]
             lib.oracle_scales_to_mma_layout.restype = None
             lib.oracle_scales_to_mma_layout.argtypes = [P, I64, I64, P]
+            lib.oracle_e4m3_value.restype = ctypes.c_double
+            lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+            lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+            lib.oracle_e4m3_encode.argtypes = [ctypes.c_double, ctypes.c_int]
+            lib.oracle_block_exponent_e4m3.restype = ctypes.c_int
+            lib.oracle_block_exponent_e4m3.argtypes = [ctypes.c_double]
+            lib.oracle_quantize_mxfp8_bf16.restype = None
+            lib.oracle_quantize_mxfp8_bf16.argtypes = [P, I64, I64, P, P]
+            lib.oracle_dequantize_mxfp8.restype = None
+            lib.oracle_dequantize_mxfp8.argtypes = [P, P, I64, I64, P]
             _lib = lib
     return _lib
 
@@ -252,3 +262,59 @@ def rfq_wgrad(x_bits: np.ndarray, dy_bits: np.ndarray, residual: bool = True, us
     dyt = np.ascontiguousarray(np.asarray(dy_bits, dtype=np.uint16).T)
     Y, S, absY = rfq_linear(xt, dyt, residual=residual, use_loops=use_loops)
     return np.ascontiguousarray(Y.T), S, np.ascontiguousarray(absY.T)
+
+
+# ----------------------------------------------------------------------------- MXFP8 comparator
+# The paper reports MXFP8 as near-lossless (abstract; section 1, first contribution)
+# and gives it as the reference point for the 4-bit formats.  OCP MX v1.0 MXFP8 with
+# E4M3 elements: 32-element blocks, E8M0 exponent floor(log2 amax) - 8, elements
+# rounded to nearest-even and saturated to +-448 (rfq_oracle.c).
+
+
+def e4m3_value(code: int) -> float:
+    """Value of one 8-bit E4M3 code (NaN for 0x7F / 0xFF)."""
+    return _load().oracle_e4m3_value(code)
+
+
+def e4m3_encode(x: float, e: int) -> int:
+    """E4M3 code of x under block exponent e (RNE on |x|*2^-e, saturate to 448, keep sign)."""
+    return _load().oracle_e4m3_encode(x, e)
+
+
+def block_exponent_e4m3(amax: float) -> int:
+    """floor(log2 amax) - 8 clamped to [-127, 127]; -127 for 0; 128 means non-finite."""
+    return _load().oracle_block_exponent_e4m3(amax)
+
+
+def quantize_mxfp8_bf16(x_bits: np.ndarray):
+    """MXFP8 quantization of a [rows, K] bf16 matrix (uint16 bit patterns): ``codes``
+    [rows, K] uint8 (one E4M3 code per element) and ``scales`` [rows, K/32] E8M0."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    rows, K = x_bits.shape
+    if K % BLOCK:
+        raise ValueError("K must be a multiple of 32")
+    out = {"codes": np.zeros((rows, K), np.uint8), "scales": np.zeros((rows, K // BLOCK), np.uint8)}
+    _load().oracle_quantize_mxfp8_bf16(_ptr(x_bits), rows, K, _ptr(out["codes"]), _ptr(out["scales"]))
+    return out
+
+
+def dequantize_mxfp8(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, K = codes.shape
+    out = np.empty((rows, K), np.float64)
+    _load().oracle_dequantize_mxfp8(_ptr(codes), _ptr(scales), rows, K, _ptr(out))
+    return out
+
+
+def mxfp8_linear(x_bits: np.ndarray, w_bits: np.ndarray, use_loops=None):
+    """Reference MXFP8 (W8A8) linear layer: Y = DQ(Q8(X)) . DQ(Q8(W))^T in float64.
+    Returns (Y, S, absY) with S = max_{i,j} sum_k |a_ik| |b_jk| as ``rfq_linear``."""
+    qa = quantize_mxfp8_bf16(x_bits)
+    qw = quantize_mxfp8_bf16(w_bits)
+    A = dequantize_mxfp8(qa["codes"], qa["scales"])
+    B = dequantize_mxfp8(qw["codes"], qw["scales"])
+    if use_loops is None:
+        use_loops = A.shape[0] * B.shape[0] * A.shape[1] <= 64 * 1024 * 1024
+    Y, absY = gemm_loops(A, B) if use_loops else gemm_blas(A, B)
+    return Y, float(absY.max()) if absY.size else 0.0, absY

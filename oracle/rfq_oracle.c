@@ -266,3 +266,106 @@ void oracle_scales_to_mma_layout(const uint8_t* plain, int64_t rows, int64_t Kb,
         for (int64_t c = 0; c < Kb; ++c)
             out[oracle_mma_scale_offset(r, c, Kb)] = plain[r * Kb + c];
 }
+
+/* ------------------------------------------------------------------------- */
+/* MXFP8 (E4M3 elements) comparator.  The paper reports MXFP8 as near-lossless
+ * (abstract; section 1, the first contribution); the format is the OCP MX v1.0
+ * MXFP8 E4M3 rule: 32-element blocks along K, E8M0 scale exponent
+ * floor(log2(amax)) - 8 (8 = the E4M3 largest exponent), elements rounded to the
+ * nearest E4M3 value with ties to even and saturated to +-448.
+ *
+ * E4M3 ("fn": no infinities): bit 7 sign, bits 6..3 exponent E (bias 7), bits 2..0
+ * mantissa m.  E == 0: subnormal 2^-6 * m/8; otherwise 2^(E-7) * (1 + m/8);
+ * E == 15 and m == 7 is NaN, so the largest finite magnitude is 2^8 * 1.75 = 448. */
+
+double oracle_e4m3_value(uint8_t code)
+{
+    int sign = (code >> 7) & 1;
+    int E = (code >> 3) & 15;
+    int m = code & 7;
+    if (E == 15 && m == 7) return NAN;
+    double mag = (E == 0) ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, E - 7);
+    return sign ? -mag : mag;
+}
+
+/* Round a non-negative real v onto the E4M3 magnitudes (codes 0x00..0x7E, which
+ * increase with the code): the nearest, ties to the even code (mantissa bit 0
+ * clear); v beyond 448 gets 448 (saturation). */
+static uint8_t e4m3_round_magnitude(double v)
+{
+    if (v >= 448.0) return 0x7E;
+    /* largest code whose value is <= v (binary search over the increasing table) */
+    int lo = 0, hi = 0x7E;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) / 2;
+        if (oracle_e4m3_value((uint8_t)mid) <= v) lo = mid; else hi = mid - 1;
+    }
+    if (lo == 0x7E) return 0x7E;
+    double below = oracle_e4m3_value((uint8_t)lo), above = oracle_e4m3_value((uint8_t)(lo + 1));
+    double db = v - below, da = above - v;
+    if (db < da) return (uint8_t)lo;
+    if (da < db) return (uint8_t)(lo + 1);
+    return (lo & 1) ? (uint8_t)(lo + 1) : (uint8_t)lo;
+}
+
+uint8_t oracle_e4m3_encode(double x, int e)
+{
+    double v = ldexp(fabs(x), -e);
+    uint8_t mag = e4m3_round_magnitude(v);
+    return (uint8_t)((signbit(x) ? 0x80 : 0x00) | mag);
+}
+
+/* floor(log2(amax)) - 8 clamped to [-127, 127]; 0 gives -127; 128 = non-finite. */
+int oracle_block_exponent_e4m3(double amax)
+{
+    if (!isfinite(amax))
+        return 128;
+    if (amax == 0.0)
+        return -127;
+    int p;
+    (void)frexp(amax, &p);
+    int e = (p - 1) - 8;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e;
+}
+
+/* MXFP8 quantization of a row-major bf16 x[rows][K]: codes [rows][K] one byte per
+ * element, scales [rows][K/32] E8M0 plain row-major.  A block holding a NaN or
+ * infinity gets scale 0xFF and codes 0 (unspecified). */
+void oracle_quantize_mxfp8_bf16(const uint16_t* x, int64_t rows, int64_t K, uint8_t* codes, uint8_t* scales)
+{
+    const int64_t Kb = K / RFQ_BLOCK;
+    for (int64_t m = 0; m < rows; ++m)
+        for (int64_t kb = 0; kb < Kb; ++kb) {
+            const uint16_t* src = x + m * K + kb * RFQ_BLOCK;
+            double v[RFQ_BLOCK], amax = 0.0;
+            int finite = 1;
+            for (int i = 0; i < RFQ_BLOCK; ++i) {
+                v[i] = oracle_bf16_value(src[i]);
+                if (!isfinite(v[i])) finite = 0;
+                if (fabs(v[i]) > amax) amax = fabs(v[i]);
+            }
+            uint8_t* dst = codes + m * K + kb * RFQ_BLOCK;
+            if (!finite) {
+                scales[m * Kb + kb] = E8M0_NAN;
+                memset(dst, 0, RFQ_BLOCK);
+                continue;
+            }
+            int e = oracle_block_exponent_e4m3(amax);
+            scales[m * Kb + kb] = (uint8_t)(e + 127);
+            for (int i = 0; i < RFQ_BLOCK; ++i) dst[i] = oracle_e4m3_encode(v[i], e);
+        }
+}
+
+/* DQ of MXFP8: out[m][k] = value(code) * 2^(scale - 127); a 0xFF scale gives NaN. */
+void oracle_dequantize_mxfp8(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K, double* out)
+{
+    const int64_t Kb = K / RFQ_BLOCK;
+    for (int64_t m = 0; m < rows; ++m)
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t s = scales[m * Kb + k / RFQ_BLOCK];
+            double val = oracle_e4m3_value(codes[m * K + k]);
+            out[m * K + k] = (s == E8M0_NAN) ? NAN : ldexp(val, (int)s - 127);
+        }
+}

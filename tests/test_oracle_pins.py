@@ -416,3 +416,78 @@ def test_oracle_shares_nothing_with_cuda_path():
             src = open(os.path.join(here, "oracle", name)).read()
             assert not re.search(r"^\s*(from|import)\s+block_scaled_gemm_rfq_b200", src, re.M), name
             assert "#include \"rfq.h\"" not in src and "csrc" not in src, name
+
+
+# --------------------------------------------------------------------------- MXFP8 comparator
+F8 = ml_dtypes.float8_e4m3fn
+
+
+def test_e4m3_decode_matches_ml_dtypes_and_torch(oracle):
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    mine = np.array([oracle.e4m3_value(int(c)) for c in codes])
+    mld = codes.view(F8).astype(np.float64)
+    tch = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(np.isnan(mine), np.isnan(mld))
+    ok = ~np.isnan(mine)
+    np.testing.assert_array_equal(mine[ok], mld[ok])
+    np.testing.assert_array_equal(mine[ok], tch[ok])
+    assert mine[0x7E] == 448.0 and math.copysign(1.0, mine[0x80]) == -1.0
+
+
+@pytest.mark.parametrize("e", [-127, -3, 0, 5, 117])
+def test_e4m3_encode_exhaustive_vs_ml_dtypes(oracle, e):
+    """Every finite bf16 x with |x| 2^-e < 512: the oracle's code equals ml_dtypes'
+    round-to-nearest-even float8_e4m3fn cast of the exactly scaled value where that
+    cast is finite (below 464); from 464 the oracle saturates to 448."""
+    _, x = _all_finite_bf16()
+    v = np.ldexp(x, -e)
+    keep = np.abs(v) < 512.0
+    x, v = x[keep], v[keep]
+    got = np.array([oracle.e4m3_encode(float(xi), e) for xi in x], dtype=np.uint8)
+    small = np.abs(v) < 464.0
+    want = v[small].astype(np.float32).astype(F8).view(np.uint8)
+    bad = np.nonzero(got[small] != want)[0]
+    assert bad.size == 0, (x[small][bad[:5]], got[small][bad[:5]], want[bad[:5]])
+    big = ~small
+    np.testing.assert_array_equal(got[big] & 0x7F, np.full(big.sum(), 0x7E, np.uint8))
+    np.testing.assert_array_equal(got[big] >> 7, (np.signbit(x[big])).astype(np.uint8))
+
+
+def test_e4m3_block_exponent_brute_force(oracle):
+    """The unique e in [-127, 127] with 256 <= amax 2^-e < 512 (E4M3's largest
+    exponent is 8), by search; -127 below the range, 128 for non-finite."""
+    rng = np.random.default_rng(21)
+    amaxes = np.concatenate([np.ldexp(rng.uniform(1, 2, 400), rng.integers(-140, 127, 400)),
+                             np.ldexp(1.0, np.arange(-130, 127)), [0.0, 448.0, 449.0, 511.9, 512.0]])
+    for a in amaxes:
+        want = -127
+        if a > 0:
+            for e in range(-127, 128):
+                if 256.0 <= math.ldexp(float(a), -e) < 512.0:
+                    want = e
+                    break
+        assert oracle.block_exponent_e4m3(float(a)) == want, a
+    assert oracle.block_exponent_e4m3(math.inf) == 128
+
+
+def test_mxfp8_qdq_identity_and_gemm_closed_form(oracle):
+    """Blocks of E4M3 values times 2^t with amax >= 256 * 2^t are reproduced exactly;
+    the MXFP8 GEMM of such operands is the plain float64 product."""
+    rng = np.random.default_rng(23)
+    vals = np.arange(0x7F, dtype=np.uint8).view(F8).astype(np.float64)     # all finite magnitudes
+    def block_matrix(rows, K):
+        m = rng.choice(vals, (rows, K)) * rng.choice([-1.0, 1.0], (rows, K))
+        m = m.reshape(rows, K // 32, 32)
+        m[:, :, 0] = rng.choice([256.0, 320.0, 448.0], (rows, K // 32))
+        m *= np.exp2(rng.integers(-30, 30, (rows, K // 32, 1)))
+        return m.reshape(rows, K)
+    X = block_matrix(48, 128)
+    W = block_matrix(40, 128)
+    xb, wb = wl.f64_to_bf16_bits(X), wl.f64_to_bf16_bits(W)
+    # every E4M3 value has <= 4 significant bits, so bf16 holds X and W exactly
+    np.testing.assert_array_equal(wl.bf16_bits_to_f32(xb).astype(np.float64), X)
+    q = oracle.quantize_mxfp8_bf16(xb)
+    np.testing.assert_array_equal(oracle.dequantize_mxfp8(q["codes"], q["scales"]), X)
+    Y, S, _ = oracle.mxfp8_linear(xb, wb)
+    np.testing.assert_allclose(Y, X @ W.T, rtol=0, atol=1e-12 * S)
