@@ -22,6 +22,7 @@ __all__ = [
     "debug_skip_next_fill", "STATIC_WORKSPACE_BYTES", "linear_fused", "linear_fused_alloc", "debug_fused_split",
     "FUSED_MAX_M", "quantize_mxfp4_t", "gemm_yt", "linear_dgrad", "linear_wgrad", "linear_wgrad_workspace_bytes",
     "quantize_mxfp4_t_alloc", "linear_wgrad_alloc", "linear_dgrad_alloc",
+    "mxfp8_codes_bytes", "quantize_mxfp8", "gemm_mxfp8", "quantize_mxfp8_alloc", "gemm_mxfp8_alloc",
     "QuantizedTensor", "quantize_mxfp4_alloc", "quantize_weight_alloc", "gemm_alloc", "linear_alloc",
     "EXPORTED_SYMBOLS", "OUT_F32", "OUT_BF16",
 ]
@@ -43,6 +44,7 @@ EXPORTED_SYMBOLS = (
     "rfq_gemm", "rfq_linear_workspace_bytes", "rfq_linear", "rfq_check_device_error", "rfq_debug_skip_next_fill",
     "rfq_linear_static_workspace", "rfq_linear_fused", "rfq_debug_fused_split", "rfq_quantize_mxfp4_t",
     "rfq_gemm_yt", "rfq_linear_dgrad", "rfq_linear_wgrad_workspace_bytes", "rfq_linear_wgrad",
+    "rfq_mxfp8_codes_bytes", "rfq_quantize_mxfp8", "rfq_gemm_mxfp8",
 )
 
 # Size of the library's fixed scratch array (RFQ_STATIC_WORKSPACE_BYTES in include/rfq.h).
@@ -91,6 +93,9 @@ def load_library():
                 "rfq_linear_dgrad": (I, [P, I64, I64, P, P, I64, P, I, I, P, SZ, P]),
                 "rfq_linear_wgrad_workspace_bytes": (SZ, [I64, I64, I64, I]),
                 "rfq_linear_wgrad": (I, [P, P, I64, I64, I64, P, I, I, P, SZ, P]),
+                "rfq_mxfp8_codes_bytes": (SZ, [I64, I64]),
+                "rfq_quantize_mxfp8": (I, [P, I64, I64, P, P, P]),
+                "rfq_gemm_mxfp8": (I, [P, P, P, P, I64, I64, I64, P, I, P]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(lib, name)
@@ -229,6 +234,25 @@ def linear_wgrad(x, dy, dw, workspace, use_residual=True, stream=None):
                                            _ptr(workspace), workspace.numel(), _stream(stream)), "rfq_linear_wgrad")
 
 
+def mxfp8_codes_bytes(rows: int, K: int) -> int:
+    return int(load_library().rfq_mxfp8_codes_bytes(rows, K))
+
+
+def quantize_mxfp8(x, codes, scales, stream=None):
+    """rfq_quantize_mxfp8: the MXFP8 (E4M3) comparator quantizer."""
+    M, K = x.shape
+    _check(load_library().rfq_quantize_mxfp8(_ptr(x), M, K, _ptr(codes), _ptr(scales), _stream(stream)),
+           "rfq_quantize_mxfp8")
+
+
+def gemm_mxfp8(qx_codes, qx_scales, qw_codes, qw_scales, M, N, K, y, stream=None):
+    """rfq_gemm_mxfp8: Y = DQ(QX) . DQ(QW)^T on kind::mxf8f6f4 MMAs."""
+    import torch
+    y_type = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
+    _check(load_library().rfq_gemm_mxfp8(_ptr(qx_codes), _ptr(qx_scales), _ptr(qw_codes), _ptr(qw_scales),
+                                         M, N, K, _ptr(y), y_type, _stream(stream)), "rfq_gemm_mxfp8")
+
+
 def check_device_error(stream=None):
     """Synchronize and report a bounded-wait timeout inside a kernel (raises RFQError)."""
     detail = ctypes.c_int(0)
@@ -325,6 +349,20 @@ def linear_wgrad_alloc(x, dy, out_dtype=None, use_residual=True, stream=None):
     ws = _empty_u8(linear_wgrad_workspace_bytes(M, K, N, use_residual), x.device)
     linear_wgrad(x, dy, dw, ws, use_residual, stream)
     return dw
+
+
+def quantize_mxfp8_alloc(x, stream=None) -> QuantizedTensor:
+    M, K = x.shape
+    q = QuantizedTensor(M, K, _empty_u8(mxfp8_codes_bytes(M, K), x.device), _empty_u8(scales_bytes(M, K), x.device))
+    quantize_mxfp8(x, q.codes, q.scales, stream)
+    return q
+
+
+def gemm_mxfp8_alloc(qa: QuantizedTensor, qw: QuantizedTensor, out_dtype=None, stream=None):
+    import torch
+    y = torch.empty((qa.rows, qw.rows), dtype=out_dtype or torch.bfloat16, device=qa.codes.device)
+    gemm_mxfp8(qa.codes, qa.scales, qw.codes, qw.scales, qa.rows, qw.rows, qa.K, y, stream)
+    return y
 
 
 def linear_alloc(x, qw: QuantizedTensor, out_dtype=None, use_residual=True, stream=None):

@@ -128,6 +128,15 @@ rfq_status_t gemm_impl(const void* qxc, const void* qxs, const void* qrc, const 
                                     y_transposed, sms, g_encode_tiled, skip, stream));
 }
 
+rfq_status_t quantize8_impl(const void* x, int64_t M, int64_t K, void* qc, void* qs, cudaStream_t stream) {
+  rfq_status_t st = check_quantize_args(x, M, K, qc, qs, nullptr, nullptr);
+  if (st != RFQ_OK) return st;
+  if (M == 0 || K == 0) return RFQ_OK;
+  int sms = 0;
+  if ((st = current_device(&sms)) != RFQ_OK) return st;
+  return from_cuda(rfq::launch_quantize_mxfp8(x, M, K, qc, qs, sms, g_encode_tiled, stream));
+}
+
 rfq_status_t quantize_t_impl(const void* x, int64_t R, int64_t C, void* qc, void* qs, void* rc, void* rs,
                              cudaStream_t stream) {
   if (R < 0 || C < 0) return RFQ_ERR_INVALID_ARG;
@@ -294,6 +303,36 @@ rfq_status_t rfq_linear_wgrad(const void* x_bf16, const void* dy_bf16, int64_t M
   if (st != RFQ_OK) return st;
   // dW^T [K][N] = (X^T)^ . (dY^T)^T, written transposed: dW [N][K]
   return gemm_impl(qxc, qxs, qrc, qrs, yt, yt + ycb, K, N, M, dw, dw_type, stream, true);
+}
+
+size_t rfq_mxfp8_codes_bytes(int64_t rows, int64_t K) {
+  if (!shape_ok(rows, K)) return 0;
+  return static_cast<size_t>(rows) * static_cast<size_t>(K);
+}
+
+rfq_status_t rfq_quantize_mxfp8(const void* x_bf16, int64_t M, int64_t K, void* q_codes, void* q_scales,
+                                cudaStream_t stream) {
+  return quantize8_impl(x_bf16, M, K, q_codes, q_scales, stream);
+}
+
+rfq_status_t rfq_gemm_mxfp8(const void* qx_codes, const void* qx_scales, const void* qw_codes, const void* qw_scales,
+                            int64_t M, int64_t N, int64_t K, void* y, rfq_out_t y_type, cudaStream_t stream) {
+  if (M < 0 || N < 0 || K < 0) return RFQ_ERR_INVALID_ARG;
+  if (y_type != RFQ_OUT_F32 && y_type != RFQ_OUT_BF16) return RFQ_ERR_INVALID_ARG;
+  if (!shape_ok(M, K) || !shape_ok(N, K) || (N % 8) != 0) return RFQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return RFQ_OK;
+  if (!y) return RFQ_ERR_INVALID_ARG;
+  if (!aligned16(y)) return RFQ_ERR_MISALIGNED;
+  int sms = 0;
+  rfq_status_t st = current_device(&sms);
+  if (st != RFQ_OK) return st;
+  const size_t y_bytes = static_cast<size_t>(M) * static_cast<size_t>(N) * (y_type == RFQ_OUT_BF16 ? 2u : 4u);
+  if (K == 0) return from_cuda(cudaMemsetAsync(y, 0, y_bytes, stream));
+  if (!qx_codes || !qx_scales || !qw_codes || !qw_scales) return RFQ_ERR_INVALID_ARG;
+  if (!aligned16(qx_codes) || !aligned16(qx_scales) || !aligned16(qw_codes) || !aligned16(qw_scales))
+    return RFQ_ERR_MISALIGNED;
+  return from_cuda(rfq::launch_gemm_mxfp8(qx_codes, qx_scales, qw_codes, qw_scales, M, N, K, y,
+                                          y_type == RFQ_OUT_BF16, sms, g_encode_tiled, stream));
 }
 
 rfq_status_t rfq_check_device_error(cudaStream_t stream, int* detail) {

@@ -119,23 +119,30 @@ __device__ __forceinline__ uint64_t scale_desc(const void* p) {
   return ((addr >> 4) & 0x3FFFull) | ((128ull >> 4) << 32) | (1ull << 46);
 }
 
-// Instruction descriptor of kind::mxf4 with E8M0 scales: E2M1 x E2M1, both
-// K-major, M = 128 * kPair, N = 256, scale-factor byte selectors for A and B.
-template <int kPair>
+// Instruction descriptor of kind::mxf4 (E2M1 x E2M1) or kind::mxf8f6f4 (E4M3 x
+// E4M3) with E8M0 scales: both K-major, M = 128 * kPair, N = 256, scale-factor
+// byte selectors for A and B.
+template <int kPair, bool kFp8>
 __device__ __forceinline__ uint32_t mma_idesc(uint32_t sf_id) {
+  constexpr uint32_t kFmt = kFp8 ? 0u : 1u;      // E4M3 in kind::mxf8f6f4, E2M1 in kind::mxf4
   return (sf_id << 4)                            // B scale-factor id
-         | (1u << 7)                             // A format E2M1
-         | (1u << 10)                            // B format E2M1
+         | (kFmt << 7)                           // A format
+         | (kFmt << 10)                          // B format
          | (uint32_t(kBN >> 3) << 17)            // N / 8
          | (1u << 23)                            // scale type UE8M0
          | (uint32_t((kBM * kPair) >> 4) << 24)  // M / 16
          | (sf_id << 29);                        // A scale-factor id
 }
 
-template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut>
+template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     rfq_gemm_kernel(const __grid_constant__ Maps maps, const GemmParams p) {
   using L = Layout<kPair>;
+  // A stage is 128 bytes of codes per row either way: 256 K of FP4 (2 scale atoms
+  // per operand row tile) or 128 K of FP8 (1 atom).
+  constexpr int kKAtoms = kFp8 ? 1 : 2;
+  constexpr uint32_t kSfaBytes = 512u * kKAtoms;        // one row tile
+  constexpr uint32_t kSfbBytes = 2u * 512u * kKAtoms;   // two row tiles (256 rows of W)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStage);
@@ -194,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int fill = 0;
       // Bytes one CTA loads per stage; the leader arms its full barrier with the
       // bytes of both CTAs of a pair (the peer's copies complete on it too).
-      const uint32_t bytes_cta = L::kATile + L::kBTile + 1024u + 2048u + (kResidual ? L::kATile + 1024u : 0u);
+      const uint32_t bytes_cta = L::kATile + L::kBTile + kSfaBytes + kSfbBytes + (kResidual ? L::kATile + kSfaBytes : 0u);
       const uint32_t bytes = bytes_cta * kPair;
       for (int tile = unit; tile < p.num_tiles; tile += num_units) {
         const int mb = tile / p.num_nb;
@@ -212,17 +219,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_2d_pair(st + L::kOffA, &maps.x, bar, kt * kBKBytes, row_a);
               if (kResidual) tma_load_2d_pair(st + L::kOffR, &maps.r, bar, kt * kBKBytes, row_a);
               tma_load_2d_pair(st + L::kOffB, &maps.w, bar, kt * kBKBytes, row_b);
-              tma_load_4d_pair(st + L::kOffSfaX, &maps.sx, bar, 0, 0, 2 * kt, rt_a);
-              if (kResidual) tma_load_4d_pair(st + L::kOffSfaR, &maps.sr, bar, 0, 0, 2 * kt, rt_a);
-              tma_load_4d_pair(st + L::kOffSfb, &maps.sw, bar, 0, 0, 2 * kt, 2 * nb);
+              tma_load_4d_pair(st + L::kOffSfaX, &maps.sx, bar, 0, 0, kKAtoms * kt, rt_a);
+              if (kResidual) tma_load_4d_pair(st + L::kOffSfaR, &maps.sr, bar, 0, 0, kKAtoms * kt, rt_a);
+              tma_load_4d_pair(st + L::kOffSfb, &maps.sw, bar, 0, 0, kKAtoms * kt, 2 * nb);
             } else {
               mbar_arrive_expect_tx(&full[stage], bytes);
               tma_load_2d(st + L::kOffA, &maps.x, &full[stage], kt * kBKBytes, row_a);
               if (kResidual) tma_load_2d(st + L::kOffR, &maps.r, &full[stage], kt * kBKBytes, row_a);
               tma_load_2d(st + L::kOffB, &maps.w, &full[stage], kt * kBKBytes, row_b);
-              tma_load_4d(st + L::kOffSfaX, &maps.sx, &full[stage], 0, 0, 2 * kt, rt_a);
-              if (kResidual) tma_load_4d(st + L::kOffSfaR, &maps.sr, &full[stage], 0, 0, 2 * kt, rt_a);
-              tma_load_4d(st + L::kOffSfb, &maps.sw, &full[stage], 0, 0, 2 * kt, 2 * nb);
+              tma_load_4d(st + L::kOffSfaX, &maps.sx, &full[stage], 0, 0, kKAtoms * kt, rt_a);
+              if (kResidual) tma_load_4d(st + L::kOffSfaR, &maps.sr, &full[stage], 0, 0, kKAtoms * kt, rt_a);
+              tma_load_4d(st + L::kOffSfb, &maps.sw, &full[stage], 0, 0, kKAtoms * kt, 2 * nb);
             }
             filled |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -264,29 +271,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint8_t* st = smem + stage * L::kStage;
           const uint32_t sf = tmem + kSfBase + stage * kSfSlot;
 #pragma unroll
-          for (uint32_t a = 0; a < 2; ++a) {
+          for (uint32_t a = 0; a < kKAtoms; ++a) {
             tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfaXCol + 4 * a, scale_desc(st + L::kOffSfaX + 512 * a));
             if (kResidual)
               tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfaRCol + 4 * a, scale_desc(st + L::kOffSfaR + 512 * a));
             tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfbCol + 8 * a, scale_desc(st + L::kOffSfb + 512 * a));
-            tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfbCol + 8 * a + 4, scale_desc(st + L::kOffSfb + 1024 + 512 * a));
+            tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfbCol + 8 * a + 4,
+                                              scale_desc(st + L::kOffSfb + 512 * kKAtoms + 512 * a));
           }
           const uint64_t da = operand_desc(st + L::kOffA);
           const uint64_t db = operand_desc(st + L::kOffB);
-          // 4 MMAs of K = 64 per operand: step q uses k-atom q/2 and scale bytes 2(q%2), 2(q%2)+1.
+          // 4 MMAs per operand over the stage's 128 bytes of K, 32 bytes each.  FP4:
+          // K = 64, step q uses k-atom q/2 and scale bytes 2(q%2), 2(q%2)+1; FP8: K = 32,
+          // step q uses scale byte q of the single k-atom.
 #pragma unroll
           for (uint32_t q = 0; q < 4; ++q) {
-            const uint32_t id = 2u * (q & 1u), a = q >> 1;
-            mma_mxf4_g<kPair>(tmem + kAccCol, da + 2u * q, db + 2u * q, mma_idesc<kPair>(id),
-                              (sf + kSfaXCol + 4 * a) | (id << 30), (sf + kSfbCol + 8 * a) | (id << 30),
-                              (kt | q) != 0 ? 1u : 0u);
+            const uint32_t id = kFp8 ? q : 2u * (q & 1u), a = kFp8 ? 0u : q >> 1;
+            const uint32_t sfa = (sf + kSfaXCol + 4 * a) | (id << 30), sfb = (sf + kSfbCol + 8 * a) | (id << 30);
+            const uint32_t acc = (kt | q) != 0 ? 1u : 0u;
+            if constexpr (kFp8)
+              mma_mxf8_g<kPair>(tmem + kAccCol, da + 2u * q, db + 2u * q, mma_idesc<kPair, true>(id), sfa, sfb, acc);
+            else
+              mma_mxf4_g<kPair>(tmem + kAccCol, da + 2u * q, db + 2u * q, mma_idesc<kPair, false>(id), sfa, sfb, acc);
           }
           if (kResidual) {
             const uint64_t dr = operand_desc(st + L::kOffR);
 #pragma unroll
             for (uint32_t q = 0; q < 4; ++q) {
               const uint32_t id = 2u * (q & 1u), a = q >> 1;
-              mma_mxf4_g<kPair>(tmem + kAccCol, dr + 2u * q, db + 2u * q, mma_idesc<kPair>(id),
+              mma_mxf4_g<kPair>(tmem + kAccCol, dr + 2u * q, db + 2u * q, mma_idesc<kPair, false>(id),
                                 (sf + kSfaRCol + 4 * a) | (id << 30), (sf + kSfbCol + 8 * a) | (id << 30), 1u);
             }
           }
@@ -391,9 +404,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut>
+template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut, bool kFp8 = false>
 cudaError_t launch_typed(const Maps& maps, const GemmParams& p, int grid, cudaStream_t stream) {
-  auto kernel = rfq_gemm_kernel<kPair, kResidual, kBf16Out, kTransOut>;
+  auto kernel = rfq_gemm_kernel<kPair, kResidual, kBf16Out, kTransOut, kFp8>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<kPair>::kSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -416,13 +429,18 @@ cudaError_t launch_typed(const Maps& maps, const GemmParams& p, int grid, cudaSt
 }
 
 template <int kPair, bool kTransOut>
-cudaError_t launch_mode(const Maps& maps, GemmParams p, int64_t M, bool residual, bool y_bf16, int num_sms,
+cudaError_t launch_mode(const Maps& maps, GemmParams p, int64_t M, bool residual, bool y_bf16, bool fp8, int num_sms,
                         cudaStream_t stream) {
   const int64_t num_mb = (M + kBM * kPair - 1) / (kBM * kPair);
   p.num_tiles = static_cast<int>(num_mb * p.num_nb);
   int units = num_sms / kPair;
   if (units > p.num_tiles) units = p.num_tiles;
   const int grid = units * kPair;
+  if constexpr (!kTransOut) {
+    if (fp8)   // the comparator path: plain MXFP8 (no residual term)
+      return y_bf16 ? launch_typed<kPair, false, true, false, true>(maps, p, grid, stream)
+                    : launch_typed<kPair, false, false, false, true>(maps, p, grid, stream);
+  }
   if (residual)
     return y_bf16 ? launch_typed<kPair, true, true, kTransOut>(maps, p, grid, stream)
                   : launch_typed<kPair, true, false, kTransOut>(maps, p, grid, stream);
@@ -430,24 +448,25 @@ cudaError_t launch_mode(const Maps& maps, GemmParams p, int64_t M, bool residual
                 : launch_typed<kPair, false, false, kTransOut>(maps, p, grid, stream);
 }
 
-}  // namespace
-
-cudaError_t launch_gemm(const void* qx_codes, const void* qx_scales, const void* qr_codes, const void* qr_scales,
-                        const void* qw_codes, const void* qw_scales, int64_t M, int64_t N, int64_t K, void* y,
-                        bool y_bf16, bool y_transposed, int num_sms, void* encode_tiled, int skip_fill,
-                        cudaStream_t stream) {
+cudaError_t launch_gemm_impl(const void* qx_codes, const void* qx_scales, const void* qr_codes, const void* qr_scales,
+                             const void* qw_codes, const void* qw_scales, int64_t M, int64_t N, int64_t K, void* y,
+                             bool y_bf16, bool y_transposed, bool fp8, int num_sms, void* encode_tiled, int skip_fill,
+                             cudaStream_t stream) {
   EncodeTiledFn encode = reinterpret_cast<EncodeTiledFn>(encode_tiled);
   const bool residual = qr_codes != nullptr;
   // CTA pairs once there are rows for both CTAs of a pair; single CTAs for short M.
   const bool pair = M > kBM;
+  const int64_t row_bytes = fp8 ? K : K / 2;
+  const uint32_t katoms = fp8 ? 1u : 2u;
   Maps maps;
-  if (!encode_codes_map(encode, &maps.x, qx_codes, M, K, kBM)) return cudaErrorInvalidValue;
-  if (!encode_codes_map(encode, &maps.w, qw_codes, N, K, pair ? kBN / 2 : kBN)) return cudaErrorInvalidValue;
-  if (!encode_scales_map(encode, &maps.sx, qx_scales, M, K, 1)) return cudaErrorInvalidValue;
-  if (!encode_scales_map(encode, &maps.sw, qw_scales, N, K, 2)) return cudaErrorInvalidValue;
+  if (!encode_code_rows_map(encode, &maps.x, qx_codes, M, row_bytes, kBM)) return cudaErrorInvalidValue;
+  if (!encode_code_rows_map(encode, &maps.w, qw_codes, N, row_bytes, pair ? kBN / 2 : kBN))
+    return cudaErrorInvalidValue;
+  if (!encode_scales_map(encode, &maps.sx, qx_scales, M, K, 1, katoms)) return cudaErrorInvalidValue;
+  if (!encode_scales_map(encode, &maps.sw, qw_scales, N, K, 2, katoms)) return cudaErrorInvalidValue;
   if (residual) {
-    if (!encode_codes_map(encode, &maps.r, qr_codes, M, K, kBM)) return cudaErrorInvalidValue;
-    if (!encode_scales_map(encode, &maps.sr, qr_scales, M, K, 1)) return cudaErrorInvalidValue;
+    if (!encode_code_rows_map(encode, &maps.r, qr_codes, M, row_bytes, kBM)) return cudaErrorInvalidValue;
+    if (!encode_scales_map(encode, &maps.sr, qr_scales, M, K, 1, katoms)) return cudaErrorInvalidValue;
   } else {
     maps.r = maps.x;
     maps.sr = maps.sx;
@@ -456,15 +475,33 @@ cudaError_t launch_gemm(const void* qx_codes, const void* qx_scales, const void*
   p.y = y;
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
-  p.num_kt = static_cast<int>((K + kBK - 1) / kBK);
+  const int64_t stage_k = fp8 ? 128 : kBK;   // 128 bytes of codes per row per stage
+  p.num_kt = static_cast<int>((K + stage_k - 1) / stage_k);
   p.num_nb = static_cast<int>((N + kBN - 1) / kBN);
   p.num_tiles = 0;
   p.skip_fill = skip_fill;
   if (y_transposed)
-    return pair ? launch_mode<2, true>(maps, p, M, residual, y_bf16, num_sms, stream)
-                : launch_mode<1, true>(maps, p, M, residual, y_bf16, num_sms, stream);
-  return pair ? launch_mode<2, false>(maps, p, M, residual, y_bf16, num_sms, stream)
-              : launch_mode<1, false>(maps, p, M, residual, y_bf16, num_sms, stream);
+    return pair ? launch_mode<2, true>(maps, p, M, residual, y_bf16, false, num_sms, stream)
+                : launch_mode<1, true>(maps, p, M, residual, y_bf16, false, num_sms, stream);
+  return pair ? launch_mode<2, false>(maps, p, M, residual, y_bf16, fp8, num_sms, stream)
+              : launch_mode<1, false>(maps, p, M, residual, y_bf16, fp8, num_sms, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const void* qx_codes, const void* qx_scales, const void* qr_codes, const void* qr_scales,
+                        const void* qw_codes, const void* qw_scales, int64_t M, int64_t N, int64_t K, void* y,
+                        bool y_bf16, bool y_transposed, int num_sms, void* encode_tiled, int skip_fill,
+                        cudaStream_t stream) {
+  return launch_gemm_impl(qx_codes, qx_scales, qr_codes, qr_scales, qw_codes, qw_scales, M, N, K, y, y_bf16,
+                          y_transposed, false, num_sms, encode_tiled, skip_fill, stream);
+}
+
+cudaError_t launch_gemm_mxfp8(const void* qx_codes, const void* qx_scales, const void* qw_codes,
+                              const void* qw_scales, int64_t M, int64_t N, int64_t K, void* y, bool y_bf16,
+                              int num_sms, void* encode_tiled, cudaStream_t stream) {
+  return launch_gemm_impl(qx_codes, qx_scales, nullptr, nullptr, qw_codes, qw_scales, M, N, K, y, y_bf16, false,
+                          true, num_sms, encode_tiled, -1, stream);
 }
 
 cudaError_t read_and_clear_device_error(unsigned int* value) {

@@ -13,6 +13,10 @@ namespace rfq {
 cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, void* qx_codes, void* qx_scales, void* qr_codes,
                             void* qr_scales, int num_sms, void* encode_tiled, cudaStream_t stream);
 
+// Kernel 1 as the MXFP8 (E4M3) comparator quantizer: codes one byte per element.
+cudaError_t launch_quantize_mxfp8(const void* x, int64_t M, int64_t K, void* codes, void* scales, int num_sms,
+                                  void* encode_tiled, cudaStream_t stream);
+
 // Kernel 1t: quantizer of X^T for a row-major X [R][C] (blocks along R).
 cudaError_t launch_quantize_t(const void* x, int64_t R, int64_t C, void* qt_codes, void* qt_scales, void* qr_codes,
                               void* qr_scales, int num_sms, void* encode_tiled, cudaStream_t stream);
@@ -31,6 +35,12 @@ cudaError_t launch_linear_fused(const void* x, int64_t M, int64_t K, const void*
                                 int64_t N, void* y, bool y_bf16, bool residual, int num_sms, void* encode_tiled,
                                 cudaStream_t stream);
 void set_fused_split_override(int split);   // 0 = automatic
+
+// The MXFP8 comparator GEMM: E4M3 codes (one byte per element) with E8M0 scales in
+// the same MMA layout, plain (no residual term).
+cudaError_t launch_gemm_mxfp8(const void* qx_codes, const void* qx_scales, const void* qw_codes,
+                              const void* qw_scales, int64_t M, int64_t N, int64_t K, void* y, bool y_bf16,
+                              int num_sms, void* encode_tiled, cudaStream_t stream);
 
 // Read and clear the device error words (GEMM and quantizer) of the current device.
 cudaError_t read_and_clear_device_error(unsigned int* value);

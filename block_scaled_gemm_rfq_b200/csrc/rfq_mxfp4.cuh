@@ -171,4 +171,42 @@ __device__ __forceinline__ void quantize_block(const uint32_t (&w)[16], uint32_t
   }
 }
 
+// ---------------------------------------------------------------- MXFP8 (comparator)
+// OCP MX v1.0 MXFP8 with E4M3 elements: E8M0 exponent floor(log2 amax) - 8 (8 = the
+// E4M3 largest exponent; 448 = 1.75 * 2^8), elements rounded to nearest even and
+// saturated to +-448.  The paper reports this format as near-lossless (abstract;
+// section 1, first contribution).
+
+// 4 fp32 values -> 4 E4M3 codes in one word (element i in byte i).
+__device__ __forceinline__ uint32_t encode4_e4m3(float a0, float a1, float a2, float a3) {
+  uint32_t out;
+  asm("{\n\t.reg .b16 h0, h1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 h0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 h1, %4, %3;\n\t"
+      "mov.b32 %0, {h0, h1};\n\t}"
+      : "=r"(out)
+      : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
+  return out;
+}
+
+// MXFP8 quantization of one 32-element bf16 block: 8 words of E4M3 codes
+// (element i in byte i%4 of word i/4) and the E8M0 byte (0xFF for a non-finite
+// block, whose codes are unspecified).  x * 2^-e is exact in fp32 (or below
+// E4M3's resolution, where it encodes to 0 either way).
+__device__ __forceinline__ void quantize_block_e4m3(const uint32_t (&w)[16], uint32_t (&codes)[8], uint32_t& s_out) {
+  const uint32_t bexp = block_amax_bits(w) >> 7;
+  const uint32_t s = bexp == 0xFFu ? 0xFFu : (bexp >= 8u ? bexp - 8u : 0u);
+  const float inv = inv_scale(s == 0xFFu ? 127u : s);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float x0, x1, x2, x3, v0, v1, v2, v3;
+    unpack_bf16x2(w[2 * k], x0, x1);
+    unpack_bf16x2(w[2 * k + 1], x2, x3);
+    mul2(v0, v1, x0, x1, inv);
+    mul2(v2, v3, x2, x3, inv);
+    codes[k] = encode4_e4m3(v0, v1, v2, v3);
+  }
+  s_out = s;
+}
+
 }  // namespace rfq

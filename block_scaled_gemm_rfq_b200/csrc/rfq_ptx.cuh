@@ -153,6 +153,18 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+// The same for 8-bit E4M3 operands with per-32-element E8M0 scales
+// (kind::mxf8f6f4, K = 32 per instruction).
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
@@ -307,6 +319,20 @@ __device__ __forceinline__ void mma_mxf4_g(uint32_t d_tmem, uint64_t adesc, uint
         : "memory");
   else
     mma_mxf4(d_tmem, adesc, bdesc, idesc, sfa_tmem, sfb_tmem, accumulate);
+}
+
+template <int kPair>
+__device__ __forceinline__ void mma_mxf8_g(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  if constexpr (kPair == 2)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+  else
+    mma_mxf8(d_tmem, adesc, bdesc, idesc, sfa_tmem, sfb_tmem, accumulate);
 }
 
 // Arrive once on `bar` (same offset) in every CTA of the pair when the tcgen05

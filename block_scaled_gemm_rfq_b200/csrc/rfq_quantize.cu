@@ -126,7 +126,7 @@ __device__ __forceinline__ void zero_scale_padding(uint8_t* sx, uint8_t* sr, uin
 // kWide: X seen as [blocks/2][128 bytes] with a 128-byte swizzle (needs an even
 // block count); otherwise as [blocks][64 bytes] with a 64-byte swizzle.  Either
 // way a lane's four 16-byte reads of its block hit distinct banks.
-template <bool kResidual, bool kWordScales, bool kWide>
+template <bool kResidual, bool kWordScales, bool kWide, bool kFp8>
 __global__ void __launch_bounds__(kThreads, RFQ_Q_CTAS_PER_SM)
     rfq_quantize_kernel(const __grid_constant__ CUtensorMap tm_x, const QuantParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -205,6 +205,18 @@ __global__ void __launch_bounds__(kThreads, RFQ_Q_CTAS_PER_SM)
       }
     }
 
+    if constexpr (kFp8) {
+      // MXFP8 comparator: 32 code bytes per block
+      uint32_t c8[8], s8;
+      quantize_block_e4m3(w, c8, s8);
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(p.qx_codes + static_cast<size_t>(gb) * 32);
+        dst[0] = make_uint4(c8[0], c8[1], c8[2], c8[3]);
+        dst[1] = make_uint4(c8[4], c8[5], c8[6], c8[7]);
+      }
+      store_scale<kWordScales>(p.qx_scales, s8, valid, row, kb, p.kb4_per_tile, lane);
+      continue;
+    }
     uint32_t cx[4], cr[4], sx, sr;
     quantize_block<kResidual>(w, cx, sx, cr, sr);
     if (valid) *reinterpret_cast<uint4*>(p.qx_codes + static_cast<size_t>(gb) * 16) = make_uint4(cx[0], cx[1], cx[2], cx[3]);
@@ -377,9 +389,9 @@ cudaError_t launch_t_typed(const CUtensorMap& tm, const QuantTParams& p, int gri
 #define RFQ_Q_WIDE 1
 #endif
 
-template <bool kResidual, bool kWord, bool kWide>
+template <bool kResidual, bool kWord, bool kWide, bool kFp8 = false>
 cudaError_t launch_typed(const CUtensorMap& tm, const QuantParams& p, int grid, cudaStream_t stream) {
-  auto kernel = rfq_quantize_kernel<kResidual, kWord, kWide>;
+  auto kernel = rfq_quantize_kernel<kResidual, kWord, kWide, kFp8>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -397,16 +409,16 @@ cudaError_t launch_typed(const CUtensorMap& tm, const QuantParams& p, int grid, 
   return cudaGetLastError();
 }
 
-template <bool kResidual, bool kWord>
+template <bool kResidual, bool kWord, bool kFp8 = false>
 cudaError_t launch_width(bool wide, const CUtensorMap& tm, const QuantParams& p, int grid, cudaStream_t stream) {
-  return wide ? launch_typed<kResidual, kWord, true>(tm, p, grid, stream)
-              : launch_typed<kResidual, kWord, false>(tm, p, grid, stream);
+  return wide ? launch_typed<kResidual, kWord, true, kFp8>(tm, p, grid, stream)
+              : launch_typed<kResidual, kWord, false, kFp8>(tm, p, grid, stream);
 }
 
 }  // namespace
 
-cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, void* qx_codes, void* qx_scales, void* qr_codes,
-                            void* qr_scales, int num_sms, void* encode_tiled, cudaStream_t stream) {
+cudaError_t launch_quantize_impl(const void* x, int64_t M, int64_t K, void* qx_codes, void* qx_scales, void* qr_codes,
+                                 void* qr_scales, bool fp8, int num_sms, void* encode_tiled, cudaStream_t stream) {
   QuantParams p;
   p.qx_codes = static_cast<uint8_t*>(qx_codes);
   p.qx_scales = static_cast<uint8_t*>(qx_scales);
@@ -441,9 +453,23 @@ cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, void* qx_codes,
   if (grid < 1) grid = 1;
   const bool word = (p.Kb % 4) == 0;
   const int g = static_cast<int>(grid);
+  if (fp8)
+    return word ? launch_width<false, true, true>(wide, tm, p, g, stream)
+                : launch_width<false, false, true>(wide, tm, p, g, stream);
   if (qr_codes)
     return word ? launch_width<true, true>(wide, tm, p, g, stream) : launch_width<true, false>(wide, tm, p, g, stream);
   return word ? launch_width<false, true>(wide, tm, p, g, stream) : launch_width<false, false>(wide, tm, p, g, stream);
+}
+
+cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, void* qx_codes, void* qx_scales, void* qr_codes,
+                            void* qr_scales, int num_sms, void* encode_tiled, cudaStream_t stream) {
+  return launch_quantize_impl(x, M, K, qx_codes, qx_scales, qr_codes, qr_scales, false, num_sms, encode_tiled,
+                              stream);
+}
+
+cudaError_t launch_quantize_mxfp8(const void* x, int64_t M, int64_t K, void* codes, void* scales, int num_sms,
+                                  void* encode_tiled, cudaStream_t stream) {
+  return launch_quantize_impl(x, M, K, codes, scales, nullptr, nullptr, true, num_sms, encode_tiled, stream);
 }
 
 cudaError_t launch_quantize_t(const void* x, int64_t R, int64_t C, void* qt_codes, void* qt_scales, void* qr_codes,

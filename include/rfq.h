@@ -280,6 +280,31 @@ rfq_status_t rfq_linear_static_workspace(const void* x_bf16, int64_t M, int64_t 
                                          cudaStream_t stream);
 
 /*
+ * MXFP8 comparator path (OCP MX v1.0 MXFP8 with E4M3 elements; the paper reports
+ * this format as near-lossless, abstract and section 1, first contribution): a
+ * reference point in accuracy and throughput for the 4-bit RFQ path.  No residual.
+ *
+ * rfq_mxfp8_codes_bytes -- rows * K (one E4M3 code byte per element); 0 for bad sizes.
+ * Scales use rfq_scales_bytes(rows, K) and the same MMA layout as MXFP4.
+ *
+ * rfq_quantize_mxfp8 -- x [M][K] bf16 (16-byte aligned, K a multiple of 32) ->
+ * codes [M][K] (element k in byte k) and E8M0 scales: exponent floor(log2 amax) - 8,
+ * elements rounded to nearest even and saturated to +-448; 0xFF for a block with a
+ * NaN or infinity.  Every byte of the scale array is written.
+ *
+ * rfq_gemm_mxfp8 -- Y = DQ(QX) . DQ(QW)^T on tcgen05 kind::mxf8f6f4 block-scaled
+ * MMAs, fp32 accumulation; operands as written by rfq_quantize_mxfp8 ([M][K] and
+ * [N][K]); y [M][N] fp32 or bf16, 16-byte aligned; N a multiple of 8.
+ */
+size_t rfq_mxfp8_codes_bytes(int64_t rows, int64_t K);
+rfq_status_t rfq_quantize_mxfp8(const void* x_bf16, int64_t M, int64_t K,
+                                void* q_codes, void* q_scales, cudaStream_t stream);
+rfq_status_t rfq_gemm_mxfp8(const void* qx_codes, const void* qx_scales,
+                            const void* qw_codes, const void* qw_scales,
+                            int64_t M, int64_t N, int64_t K,
+                            void* y, rfq_out_t y_type, cudaStream_t stream);
+
+/*
  * rfq_check_device_error -- synchronize `stream`, then read and clear the current
  * device's error word that bounded waits inside the kernels set.  Returns
  * RFQ_OK, RFQ_ERR_TIMEOUT (a wait ran out; the kernel wrote no complete result),

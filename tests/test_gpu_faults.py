@@ -1,7 +1,10 @@
 """Failure detection without a GPU fault: every spin-wait inside the GEMM is bounded.
 
 The library's test hook makes the producer of the first CTA skip one stage fill, so
-the MMA warp's wait for that stage runs out (after about 1.5 s).  The kernel then
+the MMA warp's wait for that stage runs out (after about 1.5 s).  The skipped fill
+is the last one of the CTA's only tile: the producer then has nothing left to wait
+for, so the MMA warp's wait is the one that runs out (skipping an early fill would
+also leave the producer waiting for a free stage, and either wait may expire first).  The kernel then
 records the wait in the device error word, drains its own copies and MMAs, frees its
 TMEM and returns; rfq_check_device_error reports RFQ_ERR_TIMEOUT with detail 1 (the
 stage wait) and the context stays usable: the next GEMM is correct.  Both the
@@ -27,7 +30,7 @@ def test_skipped_fill_times_out_and_context_survives(rfq, oracle, M):
     torch.cuda.synchronize()
     rfq.check_device_error()
 
-    rfq.debug_skip_next_fill(0)
+    rfq.debug_skip_next_fill(K // 256 - 1)   # the last of the tile's 256-K stage fills
     y = torch.empty((M, N), dtype=torch.float32, device="cuda")
     rfq.gemm(qa.codes, qa.scales, qa.r_codes, qa.r_scales, qw.codes, qw.scales, M, N, K, y)
     with pytest.raises(rfq.RFQError) as info:
