@@ -300,6 +300,28 @@ def time_training(rfq, wk, flush, fp4_peak, hbm_peak):
     return out
 
 
+def time_mxfp8(rfq, wk, flush, fp8_peak, hbm_peak, step):
+    """The MXFP8 comparator on the FFN workload: quantizer (X, 2 B in + 1 + 1/32 B out
+    per element) and GEMM (2 M N K flops at the FP8 rate, half the FP4 rate), beside
+    the RFQ GEMM (4 M N K at the FP4 rate: the same tensor-pipe time in theory)."""
+    import torch
+    M, K, N = wk.M, wk.K, wk.N
+    x, w = step.x, step.w
+    qa = rfq.quantize_mxfp8_alloc(x)
+    qw = rfq.quantize_mxfp8_alloc(w)
+    t = time_kernel(lambda: rfq.quantize_mxfp8(x, qa.codes, qa.scales), 20, flush)
+    qbytes = M * K * 2 + M * K + M * K // 32
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    tg = time_kernel(lambda: rfq.gemm_mxfp8(qa.codes, qa.scales, qw.codes, qw.scales, M, N, K, y), 20, flush)
+    rfq.check_device_error()
+    f = 2.0 * M * N * K
+    g_ms = statistics.mean(tg)
+    return {"quantize_x": {"us": 1e3 * statistics.mean(t), "gbs": qbytes / (statistics.mean(t) * 1e-3) / 1e9},
+            "gemm": {"us": 1e3 * g_ms, "tflops": f / (g_ms * 1e-3) / 1e12,
+                     "frac_fp8_peak": f / (g_ms * 1e-3) / 1e12 / fp8_peak,
+                     "peak_basis": "measured bf16 x 2 (nominal FP8:bf16 ratio)"}}
+
+
 def quantize_bytes(M, K, residual):
     """Algorithmic HBM bytes of the fused quantizer: read X once (2 B/elem), write codes
     (0.5 B/elem) and scales (1 B per 32 elements) per output."""
@@ -435,6 +457,7 @@ def run_cuda(args, rank, world, local):
             sweep[str(Ms)] = row
         extra["m_sweep_rfq_linear"] = sweep
         extra["training_ffn"] = time_training(rfq, wk, flush, fp4_peak, hbm_peak)
+        extra["mxfp8_ffn"] = time_mxfp8(rfq, wk, flush, fp4_peak / 2.0, hbm_peak, step)
 
     # end to end through the public API with host buffers: pinned X, W in; Y out
     xh = torch.from_numpy(wk.x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -597,6 +620,10 @@ def run_fidelity(args):
             qa = rfq.quantize_mxfp4_alloc(x, residual=res)
             xhat = rfq.gemm_alloc(qa, qe, out_dtype=torch.float32, use_residual=res)
             row[f"x_rel_err_{'rfq' if res else 'mxfp4'}"] = float(torch.linalg.norm(xhat - xf) / torch.linalg.norm(xf))
+        # MXFP8 comparator (identity exact in MXFP8 too)
+        qe8 = rfq.quantize_mxfp8_alloc(eye)
+        xhat8 = rfq.gemm_mxfp8_alloc(rfq.quantize_mxfp8_alloc(x), qe8, out_dtype=torch.float32)
+        row["x_rel_err_mxfp8"] = float(torch.linalg.norm(xhat8 - xf) / torch.linalg.norm(xf))
         if wk.w_bits is not None:
             w = to_device_bf16(wk.w_bits)
             yref = xf @ w.float().t()
@@ -605,6 +632,8 @@ def run_fidelity(args):
                 qa = rfq.quantize_mxfp4_alloc(x, residual=res)
                 y = rfq.gemm_alloc(qa, qw, out_dtype=torch.float32, use_residual=res)
                 row[f"y_rel_err_{'rfq' if res else 'mxfp4'}"] = float(torch.linalg.norm(y - yref) / torch.linalg.norm(yref))
+            y8 = rfq.gemm_mxfp8_alloc(rfq.quantize_mxfp8_alloc(x), rfq.quantize_mxfp8_alloc(w), out_dtype=torch.float32)
+            row["y_rel_err_mxfp8"] = float(torch.linalg.norm(y8 - yref) / torch.linalg.norm(yref))
         rfq.check_device_error()
         report[name] = row
     return {"fidelity": report}

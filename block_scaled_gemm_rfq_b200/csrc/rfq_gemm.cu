@@ -2,7 +2,7 @@
 //
 // "Activation Outliers Matter: Robust Recovery for Quantized Multimodal LLMs",
 // section 1 (RFQ contribution paragraph): the residual of the activation is
-// requantized and "its contribution accumulated during the GEMM".  Here
+// requantized and its product is added up inside the GEMM.  Here
 //
 //     Y = DQ(QX).DQ(QW)^T + DQ(QR).DQ(QW)^T
 //

@@ -3,8 +3,8 @@
 //
 // "Activation Outliers Matter: Robust Recovery for Quantized Multimodal LLMs",
 // section 1 (RFQ contribution paragraph): X is quantized to FP4, its residual
-// R = X - DQ(Q(X)) is quantized again and "its contribution accumulated during
-// the GEMM".  "QuaRot: Outlier-Free 4-Bit Inference in Rotated LLMs" (section 4,
+// R = X - DQ(Q(X)) is quantized again and its product added up inside the
+// GEMM.  "QuaRot: Outlier-Free 4-Bit Inference in Rotated LLMs" (section 4,
 // the fused rotate -> quantize -> low-precision matmul kernel) is prior art for
 // running the activation quantizer inside the matmul kernel.
 //

@@ -174,7 +174,7 @@ __device__ __forceinline__ void quantize_block(const uint32_t (&w)[16], uint32_t
 // ---------------------------------------------------------------- MXFP8 (comparator)
 // OCP MX v1.0 MXFP8 with E4M3 elements: E8M0 exponent floor(log2 amax) - 8 (8 = the
 // E4M3 largest exponent; 448 = 1.75 * 2^8), elements rounded to nearest even and
-// saturated to +-448.  The paper reports this format as near-lossless (abstract;
+// saturated to +-448.  The paper finds this format nearly free of accuracy loss (abstract;
 // section 1, first contribution).
 
 // 4 fp32 values -> 4 E4M3 codes in one word (element i in byte i).

@@ -3,7 +3,7 @@
 // "Activation Outliers Matter: Robust Recovery for Quantized Multimodal LLMs",
 // section 1 (RFQ contribution paragraph): X is quantized to FP4 (here MXFP4), the
 // full quantization error R = X - DQ(Q(X)) is formed, and R is quantized again by
-// the same rule ("a second low-bit quantization path").  This kernel does all of
+// the same rule (a second low-bit quantization path).  This kernel does all of
 // it in one pass over X: every bf16 element is read from HBM exactly once and the
 // codes and E8M0 scales of Q(X) and Q(R) are written once, the scales directly in
 // the layout the block-scaled tensor-core MMA consumes.  R lives only in

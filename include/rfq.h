@@ -87,8 +87,8 @@ size_t rfq_scales_bytes(int64_t rows, int64_t K);
 /*
  * rfq_quantize_mxfp4 -- the fused single-pass RFQ activation quantizer.
  * Reads X once and writes Q(X) and, when the residual pointers are given, Q(R)
- * with R = X - DQ(Q(X)) (the paper's "full quantization error" requantized by
- * "a second low-bit quantization path", section 1).
+ * with R = X - DQ(Q(X)): the whole quantization error, quantized again by a second
+ * low-bit path (section 1).
  *
  *   x_bf16              [M][K] bf16, 16-byte aligned
  *   qx_codes, qx_scales Q(X): rfq_codes_bytes(M, K) and rfq_scales_bytes(M, K) bytes
@@ -114,8 +114,8 @@ rfq_status_t rfq_quantize_weight(const void* w_bf16, int64_t N, int64_t K,
 /*
  * rfq_gemm -- the RFQ GEMM: Y = DQ(QX).DQ(QW)^T + DQ(QR).DQ(QW)^T, both terms
  * accumulated in fp32 into one accumulator (equivalently one GEMM over the
- * concatenated K, [QX | QR] against [QW | QW]); "requantize the activation
- * residual during GEMM and accumulate its contribution" (section 1).
+ * concatenated K, [QX | QR] against [QW | QW]): the residual's product is added
+ * inside the GEMM (section 1).
  * qr_codes == qr_scales == NULL gives the plain MXFP4 GEMM (residual path off).
  *
  *   qx_*, qr_*   [M][K] operands as written by rfq_quantize_mxfp4
@@ -165,7 +165,7 @@ size_t rfq_linear_workspace_bytes(int64_t M, int64_t K, int use_residual);
 /*
  * rfq_linear -- the RFQ linear layer: rfq_quantize_mxfp4 of X into the caller's
  * workspace, then rfq_gemm against the pre-quantized weight, on one stream
- * ("requires no architectural modifications": a drop-in for the layer's GEMM).
+ * (the method leaves the network unchanged: a drop-in for the layer's GEMM).
  * For 1 <= M <= RFQ_FUSED_MAX_M it runs rfq_linear_fused instead (same
  * arguments checked; the workspace is then left untouched).
  *
@@ -225,8 +225,8 @@ rfq_status_t rfq_linear_wgrad(const void* x_bf16, const void* dy_bf16, int64_t M
 /*
  * rfq_linear_fused -- the RFQ linear layer in one kernel for short batches
  * (M <= RFQ_FUSED_MAX_M): the quantizer runs inside the GEMM kernel, so Q(X)
- * and Q(R) exist only in shared memory ("requantize the activation residual
- * during GEMM", section 1).  Same codes, scales and accumulation as rfq_linear;
+ * and Q(R) exist only in shared memory (the residual is requantized inside the
+ * GEMM, section 1).  Same codes, scales and accumulation as rfq_linear;
  * K is split across a cluster of CTAs per 128 columns of Y and the partial
  * sums are added in a fixed order, so Y differs from rfq_linear's only by fp32
  * summation order.  Needs no workspace.
@@ -281,7 +281,8 @@ rfq_status_t rfq_linear_static_workspace(const void* x_bf16, int64_t M, int64_t 
 
 /*
  * MXFP8 comparator path (OCP MX v1.0 MXFP8 with E4M3 elements; the paper reports
- * this format as near-lossless, abstract and section 1, first contribution): a
+ * this format as nearly free of accuracy loss, abstract and section 1, first
+ * contribution): a
  * reference point in accuracy and throughput for the 4-bit RFQ path.  No residual.
  *
  * rfq_mxfp8_codes_bytes -- rows * K (one E4M3 code byte per element); 0 for bad sizes.

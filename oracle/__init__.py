@@ -232,8 +232,8 @@ def rfq_linear(x_bits: np.ndarray, w_bits: np.ndarray, residual: bool = True, us
 
 
 # ----------------------------------------------------------------------------- backward GEMMs
-# The paper frames RFQ as aware of FP4 *training* (section 1, the RFQ paragraph:
-# "fully differentiable and training-aware") but states no backward rule.  The
+# The paper frames RFQ as a differentiable method meant for FP4 *training* (section 1,
+# the RFQ paragraph) but states no backward rule.  The
 # plainest reading is the straight-through estimator: the quantizers pass the
 # gradient unchanged, and the two backward GEMMs of Y = X W^T are themselves run on
 # MXFP4 operands quantized along *their* contraction axis, with the residual
@@ -265,7 +265,7 @@ def rfq_wgrad(x_bits: np.ndarray, dy_bits: np.ndarray, residual: bool = True, us
 
 
 # ----------------------------------------------------------------------------- MXFP8 comparator
-# The paper reports MXFP8 as near-lossless (abstract; section 1, first contribution)
+# The paper finds MXFP8 nearly free of accuracy loss (abstract; section 1, first contribution)
 # and gives it as the reference point for the 4-bit formats.  OCP MX v1.0 MXFP8 with
 # E4M3 elements: 32-element blocks, E8M0 exponent floor(log2 amax) - 8, elements
 # rounded to nearest-even and saturated to +-448 (rfq_oracle.c).

@@ -268,7 +268,7 @@ void oracle_scales_to_mma_layout(const uint8_t* plain, int64_t rows, int64_t Kb,
 }
 
 /* ------------------------------------------------------------------------- */
-/* MXFP8 (E4M3 elements) comparator.  The paper reports MXFP8 as near-lossless
+/* MXFP8 (E4M3 elements) comparator.  The paper finds MXFP8 nearly free of accuracy loss
  * (abstract; section 1, the first contribution); the format is the OCP MX v1.0
  * MXFP8 E4M3 rule: 32-element blocks along K, E8M0 scale exponent
  * floor(log2(amax)) - 8 (8 = the E4M3 largest exponent), elements rounded to the
