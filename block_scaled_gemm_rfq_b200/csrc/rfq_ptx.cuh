@@ -252,8 +252,13 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // Arrive on an mbarrier of another CTA of the cluster (shared::cluster address).
+// Release at CTA scope: the arrive orders this thread's tcgen05 accesses, which
+// tcgen05.wait / tcgen05.fence::before_thread_sync have already completed and
+// fenced; a cluster-scope release would also wait (measured ~1 us) for every
+// earlier memory operation of the thread to become visible across the cluster,
+// which nothing that waits on these barriers reads.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_address) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_address) : "memory");
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_address) : "memory");
 }
 
 // Tensor TMA load whose completion is signalled on the mbarrier at `mbar_cluster`,
