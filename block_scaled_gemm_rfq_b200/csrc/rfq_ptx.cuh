@@ -53,7 +53,7 @@ __device__ __forceinline__ bool mbar_test_parity(uint32_t bar, uint32_t parity) 
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
       : "r"(bar), "r"(parity)
@@ -61,6 +61,11 @@ __device__ __forceinline__ bool mbar_test_parity(uint32_t bar, uint32_t parity) 
   return done != 0;
 }
 
+// Acquire at CTA scope: what a completed phase hands over is shared memory written
+// by TMA (made visible by the transaction count itself) or tensor-memory state
+// ordered by tcgen05 fences, never generic stores of another CTA; a cluster-scope
+// acquire measured ~4 % slower on the GEMM mainloop, which waits once per stage.
+//
 // Wait until the phase with the given parity of `bar` has completed.  Bounded:
 // returns false (after recording `err` in *error_word and raising the
 // CTA's abort flag) when the wait runs past kWaitLimitNs, or as soon as another
