@@ -437,9 +437,11 @@ def run_cuda(args, rank, world, local):
                 cell = {"us": 1e3 * statistics.mean(t),
                         "tflops_useful": 2.0 * Ms * sk.N * sk.K / (statistics.mean(t) * 1e-3) / 1e12,
                         "us_stream": 1e3 * t_stream, "stream_sets": n_sets,
-                        "path": "fused" if Ms <= rfq.FUSED_MAX_M else "quantize+gemm"}
+                        "path": "fused" if Ms <= 32 else
+                                ("quantize+split-K gemm" if Ms <= 256 and (1 if Ms <= 128 else 2) * ((sk.N + 255) // 256)
+                                 < torch.cuda.get_device_properties(0).multi_processor_count // 2 else "quantize+gemm")}
                 if Ms <= rfq.FUSED_MAX_M:
-                    # the two-kernel path on the same problem, for comparison
+                    # the two-kernel path (quantize, then GEMM) on the same problem, for comparison
                     s2 = RfqStep(rfq, xs, ws, residual=res)
                     s2.quantize_w()
                     t2 = time_kernel(lambda: (s2.quantize_x(), s2.gemm()), 20, flush)

@@ -124,6 +124,12 @@ rfq_status_t gemm_impl(const void* qxc, const void* qxs, const void* qrc, const 
       (qrc && (!aligned16(qrc) || !aligned16(qrs))))
     return RFQ_ERR_MISALIGNED;
   const int skip = g_skip_fill.exchange(-1);
+  // Short batches whose tiles would fill less than half the SMs (M <= 128: one
+  // CTA per 256 columns; M <= 256: one CTA pair) go to the split-K kernel.
+  const int64_t tile_ctas = (M <= 128 ? 1 : 2) * ((N + 255) / 256);
+  if (!y_transposed && M <= rfq::kShortGemmMaxM && tile_ctas < sms / 2)
+    return from_cuda(rfq::launch_gemm_short(qxc, qxs, qrc, qrs, qwc, qws, M, N, K, y, y_type == RFQ_OUT_BF16, sms,
+                                            g_encode_tiled, skip, stream));
   return from_cuda(rfq::launch_gemm(qxc, qxs, qrc, qrs, qwc, qws, M, N, K, y, y_type == RFQ_OUT_BF16,
                                     y_transposed, sms, g_encode_tiled, skip, stream));
 }
@@ -234,7 +240,10 @@ rfq_status_t rfq_linear(const void* x_bf16, int64_t M, int64_t K, const void* qw
   if (K > 0 && (workspace == nullptr || workspace_bytes < need)) return RFQ_ERR_WORKSPACE;
   if (K > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return RFQ_ERR_MISALIGNED;
   if (K > 0 && (!x_bf16 || !qw_codes || !qw_scales)) return RFQ_ERR_INVALID_ARG;
-  if (M <= RFQ_FUSED_MAX_M) return fused_impl(x_bf16, M, K, qw_codes, qw_scales, N, y, y_type, use_residual, stream);
+  // Up to 32 rows the single kernel wins; from ~48 rows its repeated quantization
+  // of X per weight tile costs more than the quantizer launch it saves, and the
+  // quantizer + split-K short-batch GEMM pair is as fast or faster (measured).
+  if (M <= 32) return fused_impl(x_bf16, M, K, qw_codes, qw_scales, N, y, y_type, use_residual, stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t cb = align256(rfq_codes_bytes(M, K));
   const size_t sb = align256(rfq_scales_bytes(M, K));

@@ -36,6 +36,14 @@ cudaError_t launch_linear_fused(const void* x, int64_t M, int64_t K, const void*
                                 cudaStream_t stream);
 void set_fused_split_override(int split);   // 0 = automatic
 
+// The same kernel for pre-quantized operands (M <= 256): Q(X), Q(R) as written by
+// the quantizer come in by TMA; the GEMM's M <= 256 path when its tiles are few.
+cudaError_t launch_gemm_short(const void* qx_codes, const void* qx_scales, const void* qr_codes,
+                              const void* qr_scales, const void* qw_codes, const void* qw_scales, int64_t M,
+                              int64_t N, int64_t K, void* y, bool y_bf16, int num_sms, void* encode_tiled,
+                              int skip_fill, cudaStream_t stream);
+constexpr int64_t kShortGemmMaxM = 256;
+
 // The MXFP8 comparator GEMM: E4M3 codes (one byte per element) with E8M0 scales in
 // the same MMA layout, plain (no residual term).
 cudaError_t launch_gemm_mxfp8(const void* qx_codes, const void* qx_scales, const void* qw_codes,

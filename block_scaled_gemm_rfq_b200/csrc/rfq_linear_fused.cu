@@ -59,40 +59,49 @@ constexpr int kBKBytes = kBK / 2;         // 128 bytes of codes per row per stag
 constexpr int kQWarps = 8;                // quantizer warps, then epilogue warps
 constexpr int kQThreads = kQWarps * 32;
 constexpr int kThreads = 64 + kQThreads;  // warp 0 TMA, warp 1 MMA, warps 2..9 quantize + epilogue
-constexpr int kMaxStages = 4;
 constexpr int kMaxSplit = 8;              // portable cluster size
 constexpr int kMaxDevices = 64;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kSfBase = 128;         // accumulator: columns [0, Mp); scale slots from column 128
-constexpr uint32_t kSfSlot = 32;          // per stage: +0 QW (2 k-atoms), +8 QX, +16 QR
-constexpr uint32_t kSfW = 0, kSfX = 8, kSfR = 16;
 constexpr unsigned int kErrWaitQuantX = 7;   // a quantizer warp waiting for its staged X
 
-// Shared memory of one CTA for at most kCap rows of X (kCap = 32 or 64).
-template <int kCap>
+// Shared memory and tensor memory of one CTA for at most kCap rows of X.
+//   kPreQ = false (kCap = 32 or 64): X arrives as bf16 and the quantizer warps
+//     write Q(X), Q(R) into the stage;
+//   kPreQ = true (kCap = 256): Q(X), Q(R) codes and scale atoms, written before by
+//     the stand-alone quantizer, arrive by TMA like the weight tile (the
+//     short-batch GEMM: 64 < M <= 256, or any rfq_gemm call with few tiles).
+template <int kCap, bool kPreQ>
 struct FusedLayout {
-  static constexpr int kStages = kCap <= 32 ? 4 : 3;
-  static constexpr uint32_t kBoxBytes = kCap * 128;                // one staged box: kCap rows x 64 bf16
-  static constexpr uint32_t kOffW = 0;                             // 128 x 128 B of weight codes
-  static constexpr uint32_t kOffXs = kOffW + kBN * kBKBytes;       // staged X: 4 boxes
-  static constexpr uint32_t kOffX = kOffXs + 4 * kBoxBytes;        // Q(X) codes: kCap x 128 B
-  static constexpr uint32_t kOffR = kOffX + kCap * kBKBytes;       // Q(R) codes
-  static constexpr uint32_t kOffSfw = kOffR + kCap * kBKBytes;     // 2 scale atoms of 512 B each
-  static constexpr uint32_t kOffSfx = kOffSfw + 1024;
-  static constexpr uint32_t kOffSfr = kOffSfx + 1024;
-  static constexpr uint32_t kStage = kOffSfr + 1024;
-  // The split-K partial tile ([kCap][128] fp32) reuses stage 0's staged X,
-  // which is dead once the accumulator is complete.
-  static constexpr uint32_t kOffRed = kOffXs;
+  static constexpr int kRowTiles = (kCap + 127) / 128;               // 128-row scale atoms of the activation
+  static constexpr int kStages = kPreQ ? 2 : (kCap <= 32 ? 4 : 3);
+  static constexpr uint32_t kBoxBytes = kPreQ ? 0 : kCap * 128;      // one staged box: kCap rows x 64 bf16
+  static constexpr uint32_t kOffW = 0;                               // 128 x 128 B of weight codes
+  static constexpr uint32_t kOffXs = kOffW + kBN * kBKBytes;         // staged X: 4 boxes (kPreQ: none)
+  static constexpr uint32_t kOffX = kOffXs + 4 * kBoxBytes;          // Q(X) codes: kCap x 128 B
+  static constexpr uint32_t kOffR = kOffX + kCap * kBKBytes;         // Q(R) codes
+  static constexpr uint32_t kOffSfw = kOffR + kCap * kBKBytes;       // 2 k-atoms of 512 B
+  static constexpr uint32_t kOffSfx = kOffSfw + 1024;                // [row tile][k-atom] atoms of 512 B
+  static constexpr uint32_t kOffSfr = kOffSfx + 1024 * kRowTiles;
+  static constexpr uint32_t kStage = kOffSfr + 1024 * kRowTiles;
+  // The split-K partial tile ([kCap][128] fp32) reuses stage 0's staged X, or,
+  // with kPreQ, the ring: both are dead once the accumulator is complete.
+  static constexpr uint32_t kOffRed = kPreQ ? 0 : kOffXs;
   static constexpr uint32_t kOffBar = kStages * kStage;
   static constexpr uint32_t kSmem = kOffBar + 256 + 1024;
+  // Tensor memory: the accumulator in columns [0, Mp), then one scale slot per
+  // stage: +0 QW (2 k-atoms x 4 columns), +kSfX QX and +kSfR QR (2 k-atoms x
+  // kRowTiles x 4 columns each; k-atom a, row tile t at (a * kRowTiles + t) * 4).
+  static constexpr uint32_t kSfBase = kPreQ ? 256 : 128;
+  static constexpr uint32_t kSfSlot = kPreQ ? 64 : 32;
+  static constexpr uint32_t kSfW = 0, kSfX = 8, kSfR = 8 + 8 * kRowTiles;
+  static constexpr uint32_t kTmemCols = kPreQ ? 512 : 256;
   // Per thread and round: blocks (kCap rows x 8 blocks of one stage, or two
   // stages of 16 rows) over kQThreads threads.
   static constexpr int kSlots = kCap * 8 / kQThreads > 0 ? kCap * 8 / kQThreads : 1;
-  static_assert(kCap * kBN * 4 <= 4 * kBoxBytes, "partial tile must fit the staged X of a stage");
+  static_assert(kOffRed + kCap * kBN * 4 <= (kPreQ ? kStages * kStage : kStage), "partial tile must fit");
   static_assert(kStage % 1024 == 0 && kBoxBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
   static_assert(kSmem <= 232448, "exceeds the 227 KiB shared-memory limit");
-  static_assert(kSfBase + kMaxStages * kSfSlot <= kTmemCols, "scale slots exceed TMEM");
+  static_assert(kSfR + 8 * kRowTiles <= kSfSlot, "scale slot too small");
+  static_assert(kSfBase >= kCap && kSfBase + kStages * kSfSlot <= kTmemCols, "scale slots exceed TMEM");
   static_assert((4 * kStages + 2) * 8 + 8 <= 256, "barrier area too small");
 };
 
@@ -106,12 +115,16 @@ struct FusedParams {
   int num_kt;          // k-tiles of 256
   int group;           // k-tiles quantized per round
   uint32_t idesc_n;    // (Mp / 8) << 17
+  uint32_t act_bytes;  // kPreQ: bytes of Q(X) [+ Q(R)] codes and scale atoms per stage
+  int skip_fill;       // kPreQ fault injection: CTA (0, 0) skips this stage fill (-1 = off)
 };
 
 struct FusedMaps {
   CUtensorMap x;       // bf16 [M][K], box 64 elements x Mp rows, 128-byte swizzle, zero fill
   CUtensorMap w;       // codes [N][K/2], box 128 B x 128 rows, 128-byte swizzle
   CUtensorMap sw;      // scales [row tiles][k atoms][2][256 B], box 2 k-atoms x 1 row tile
+  CUtensorMap qx, qr;  // kPreQ: codes [M][K/2], box 128 B x Mp rows, 128-byte swizzle
+  CUtensorMap sx, sr;  // kPreQ: scales, box 2 k-atoms x ceil(Mp / 128) row tiles
 };
 
 __device__ __forceinline__ uint64_t operand_desc(const void* p) {
@@ -129,10 +142,10 @@ __device__ __forceinline__ uint32_t fused_idesc(uint32_t idesc_n, uint32_t sf_id
   return (sf_id << 4) | (1u << 7) | (1u << 10) | idesc_n | (1u << 23) | (uint32_t(kBN >> 4) << 24) | (sf_id << 29);
 }
 
-template <int kCap, bool kResidual, bool kBf16Out>
+template <int kCap, bool kResidual, bool kBf16Out, bool kPreQ>
 __global__ void __launch_bounds__(kThreads, 1)
     rfq_linear_fused_kernel(const __grid_constant__ FusedMaps maps, const FusedParams p) {
-  using L = FusedLayout<kCap>;
+  using L = FusedLayout<kCap, kPreQ>;
   constexpr int kStages = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -166,11 +179,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t phase = static_cast<uint32_t>(i / kStages) & 1u;
     uint8_t* st = smem + stage * L::kStage;
     const int kt = kt0 + i;
-    mbar_arrive_expect_tx(&xfull[stage], x_bytes);
+    if constexpr (kPreQ) {
+      if (i == p.skip_fill && blockIdx.x == 0 && blockIdx.y == 0) return;   // fault injection (tests)
+      // weight tile and the activation's codes and scale atoms, all on one barrier
+      mbar_arrive_expect_tx(&wfull[stage], kBN * kBKBytes + 1024u + p.act_bytes);
+      tma_load_2d(st + L::kOffX, &maps.qx, &wfull[stage], kt * kBKBytes, 0);
+      tma_load_4d(st + L::kOffSfx, &maps.sx, &wfull[stage], 0, 0, 2 * kt, 0);
+      if (kResidual) {
+        tma_load_2d(st + L::kOffR, &maps.qr, &wfull[stage], kt * kBKBytes, 0);
+        tma_load_4d(st + L::kOffSfr, &maps.sr, &wfull[stage], 0, 0, 2 * kt, 0);
+      }
+    } else {
+      mbar_arrive_expect_tx(&xfull[stage], x_bytes);
 #pragma unroll
-    for (int b = 0; b < 4; ++b)
-      tma_load_2d(st + L::kOffXs + b * L::kBoxBytes, &maps.x, &xfull[stage], kt * kBK + 64 * b, 0);
-    mbar_arrive_expect_tx(&wfull[stage], kBN * kBKBytes + 1024u);
+      for (int b = 0; b < 4; ++b)
+        tma_load_2d(st + L::kOffXs + b * L::kBoxBytes, &maps.x, &xfull[stage], kt * kBK + 64 * b, 0);
+      mbar_arrive_expect_tx(&wfull[stage], kBN * kBKBytes + 1024u);
+    }
     tma_load_2d(st + L::kOffW, &maps.w, &wfull[stage], kt * kBKBytes, n0);
     tma_load_4d(st + L::kOffSfw, &maps.sw, &wfull[stage], 0, 0, 2 * kt, tile);
     filled |= 1u << stage;
@@ -188,14 +213,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    prefetch_tmap(&maps.x);
+    if constexpr (kPreQ) {
+      prefetch_tmap(&maps.qx);
+      prefetch_tmap(&maps.sx);
+      if (kResidual) {
+        prefetch_tmap(&maps.qr);
+        prefetch_tmap(&maps.sr);
+      }
+    } else {
+      prefetch_tmap(&maps.x);
+    }
     prefetch_tmap(&maps.w);
     prefetch_tmap(&maps.sw);
     griddep_wait();   // X and QW may be written by the previous kernel on the stream
     for (; issued < nk && issued < kStages; ++issued) issue_stage(issued);   // the stages start free
   }
   if (warp == 1) {
-    tmem_alloc_g<1>(tmem_slot, kTmemCols);
+    tmem_alloc_g<1>(tmem_slot, L::kTmemCols);
     tmem_relinquish_g<1>();
   }
   tc_fence_before();
@@ -205,6 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   griddep_launch_dependents();
   griddep_wait();   // Y may still be read by the previous kernel on the stream
+  bool epi_ok = false;   // epilogue warps: the accumulator is complete
 
   if (warp == 0) {
     if (lane == 0) {
@@ -221,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kStages; ++s)
           if (filled & (1u << s)) {
             int never = 0;
-            mbar_wait(&xfull[s], (last_parity >> s) & 1u, &never, &g_fused_error, kErrWaitDrain);
+            if (!kPreQ) mbar_wait(&xfull[s], (last_parity >> s) & 1u, &never, &g_fused_error, kErrWaitDrain);
             mbar_wait(&wfull[s], (last_parity >> s) & 1u, &never, &g_fused_error, kErrWaitDrain);
           }
     }
@@ -233,18 +268,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int stage = i % kStages;
         const uint32_t phase = static_cast<uint32_t>(i / kStages) & 1u;
         if (!mbar_wait(&wfull[stage], phase, abort_flag, &g_fused_error, kErrWaitFull) ||
-            !mbar_wait(&qfull[stage], phase, abort_flag, &g_fused_error, kErrWaitFull)) {
+            (!kPreQ && !mbar_wait(&qfull[stage], phase, abort_flag, &g_fused_error, kErrWaitFull))) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint8_t* st = smem + stage * L::kStage;
-        const uint32_t sf = tmem + kSfBase + stage * kSfSlot;
+        const uint32_t sf = tmem + L::kSfBase + stage * L::kSfSlot;
+        constexpr uint32_t kSfW = L::kSfW, kSfX = L::kSfX, kSfR = L::kSfR, kRT = L::kRowTiles;
 #pragma unroll
         for (uint32_t a = 0; a < 2; ++a) {
           tmem_copy_32x128b_warpx4_g<1>(sf + kSfW + 4 * a, scale_desc(st + L::kOffSfw + 512 * a));
-          tmem_copy_32x128b_warpx4_g<1>(sf + kSfX + 4 * a, scale_desc(st + L::kOffSfx + 512 * a));
-          if (kResidual) tmem_copy_32x128b_warpx4_g<1>(sf + kSfR + 4 * a, scale_desc(st + L::kOffSfr + 512 * a));
+#pragma unroll
+          for (uint32_t t = 0; t < kRT; ++t) {
+            // smem atom (row tile t, k-atom a) at (2t + a) * 512 -> columns (a * kRT + t) * 4
+            tmem_copy_32x128b_warpx4_g<1>(sf + kSfX + 4 * (a * kRT + t), scale_desc(st + L::kOffSfx + 512 * (2 * t + a)));
+            if (kResidual)
+              tmem_copy_32x128b_warpx4_g<1>(sf + kSfR + 4 * (a * kRT + t),
+                                            scale_desc(st + L::kOffSfr + 512 * (2 * t + a)));
+          }
         }
         const uint64_t dw = operand_desc(st + L::kOffW);
         const uint64_t dx = operand_desc(st + L::kOffX);
@@ -253,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (uint32_t q = 0; q < 4; ++q) {
           const uint32_t id = 2u * (q & 1u), a = q >> 1;
           mma_mxf4(tmem, dw + 2u * q, dx + 2u * q, fused_idesc(p.idesc_n, id), (sf + kSfW + 4 * a) | (id << 30),
-                   (sf + kSfX + 4 * a) | (id << 30), (i | static_cast<int>(q)) != 0 ? 1u : 0u);
+                   (sf + kSfX + 4 * kRT * a) | (id << 30), (i | static_cast<int>(q)) != 0 ? 1u : 0u);
         }
         if (kResidual) {
           const uint64_t dr = operand_desc(st + L::kOffR);
@@ -261,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (uint32_t q = 0; q < 4; ++q) {
             const uint32_t id = 2u * (q & 1u), a = q >> 1;
             mma_mxf4(tmem, dw + 2u * q, dr + 2u * q, fused_idesc(p.idesc_n, id), (sf + kSfW + 4 * a) | (id << 30),
-                     (sf + kSfR + 4 * a) | (id << 30), 1u);
+                     (sf + kSfR + 4 * kRT * a) | (id << 30), 1u);
           }
         }
         tc_commit(&empty[stage]);
@@ -287,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // distinct bank groups, and write 8 distinct chunks of the B tile.
     const int qt = threadIdx.x - 64;
     const int blocks_per_stage = 8 * p.Mp;
-    const int rounds = (nk + p.group - 1) / p.group;
+    const int rounds = kPreQ ? 0 : (nk + p.group - 1) / p.group;   // kPreQ: nothing to quantize
     bool ok = true;
     for (int r = 0; r < rounds && ok; ++r) {
       const int i0 = r * p.group;
@@ -344,8 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- epilogue
     // Warp w reads TMEM lanes 32 (w % 4) .. +31 (weight rows = columns of Y);
     // the two warps of a lane quadrant alternate over 8-column chunks (rows of X).
-    ok = mbar_wait(acc_full, 0, abort_flag, &g_fused_error, kErrWaitAccFull);
-    if (__all_sync(0xffffffffu, ok)) {
+    // With a K split the accumulator goes, as [Mp][128] fp32, to this CTA's
+    // receive area for the cluster reduction below.
+    epi_ok = mbar_wait(acc_full, 0, abort_flag, &g_fused_error, kErrWaitAccFull);
+    if (__all_sync(0xffffffffu, epi_ok)) {
       tc_fence_after();
       const int quad = warp & 3;
       const int half = (warp - 2) >> 2;
@@ -378,7 +422,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the error path too.  After the first, CTA s sums its 1/S of the tile over
     // the cluster's partials in rank order (into registers); it arrives on the
     // second as soon as its reads of the peers are done and stores Y while the
-    // others finish theirs.
+    // others finish theirs.  (Pushing the partials to their owners with 4-byte
+    // distributed stores instead measured slower; the exchange is bound by the
+    // distributed shared-memory bandwidth either way.)
     cluster_sync();
     constexpr int kPer = kCap / 16;            // >= ceil(F / split / kQThreads) for split >= 2
     float4 acc[kPer];
@@ -430,16 +476,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc_g<1>(tmem, kTmemCols);
+    tmem_dealloc_g<1>(tmem, L::kTmemCols);
   }
 }
 
 std::atomic<int> g_split_override{0};
 
-template <int kCap, bool kResidual, bool kBf16Out>
+template <int kCap, bool kResidual, bool kBf16Out, bool kPreQ = false>
 cudaError_t launch_typed(const FusedMaps& maps, const FusedParams& p, int tiles, int num_sms, cudaStream_t stream) {
-  using L = FusedLayout<kCap>;
-  auto kernel = rfq_linear_fused_kernel<kCap, kResidual, kBf16Out>;
+  using L = FusedLayout<kCap, kPreQ>;
+  auto kernel = rfq_linear_fused_kernel<kCap, kResidual, kBf16Out, kPreQ>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -537,9 +583,55 @@ cudaError_t launch_linear_fused(const void* x, int64_t M, int64_t K, const void*
   p.group = p.Mp * 8 >= kQThreads ? 1 : kQThreads / (p.Mp * 8);
   if (p.group > 3) p.group = 3;   // <= the stages of either layout
   p.idesc_n = static_cast<uint32_t>(p.Mp >> 3) << 17;
+  p.act_bytes = 0;
+  p.skip_fill = -1;
+  maps.qx = maps.qr = maps.w;   // unused without kPreQ
+  maps.sx = maps.sr = maps.sw;
   const int tiles = static_cast<int>((N + kBN - 1) / kBN);
   return p.Mp <= 32 ? launch_cap<32>(maps, p, tiles, residual, y_bf16, num_sms, stream)
                     : launch_cap<64>(maps, p, tiles, residual, y_bf16, num_sms, stream);
+}
+
+cudaError_t launch_gemm_short(const void* qx_codes, const void* qx_scales, const void* qr_codes,
+                              const void* qr_scales, const void* qw_codes, const void* qw_scales, int64_t M,
+                              int64_t N, int64_t K, void* y, bool y_bf16, int num_sms, void* encode_tiled,
+                              int skip_fill, cudaStream_t stream) {
+  EncodeTiledFn encode = reinterpret_cast<EncodeTiledFn>(encode_tiled);
+  const bool residual = qr_codes != nullptr;
+  const int64_t Mp = (M + 15) / 16 * 16;
+  const uint32_t row_tiles = static_cast<uint32_t>((Mp + 127) / 128);
+  FusedMaps maps;
+  if (!encode_codes_map(encode, &maps.w, qw_codes, N, K, kBN)) return cudaErrorInvalidValue;
+  if (!encode_scales_map(encode, &maps.sw, qw_scales, N, K, 1)) return cudaErrorInvalidValue;
+  if (!encode_codes_map(encode, &maps.qx, qx_codes, M, K, static_cast<uint32_t>(Mp))) return cudaErrorInvalidValue;
+  if (!encode_scales_map(encode, &maps.sx, qx_scales, M, K, row_tiles)) return cudaErrorInvalidValue;
+  if (residual) {
+    if (!encode_codes_map(encode, &maps.qr, qr_codes, M, K, static_cast<uint32_t>(Mp))) return cudaErrorInvalidValue;
+    if (!encode_scales_map(encode, &maps.sr, qr_scales, M, K, row_tiles)) return cudaErrorInvalidValue;
+  } else {
+    maps.qr = maps.qx;
+    maps.sr = maps.sx;
+  }
+  maps.x = maps.w;   // unused with kPreQ
+  FusedParams p;
+  p.y = y;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.Kb = static_cast<int>(K / 32);
+  p.Mp = static_cast<int>(Mp);
+  p.num_kt = static_cast<int>((K + kBK - 1) / kBK);
+  p.group = 1;
+  p.idesc_n = static_cast<uint32_t>(p.Mp >> 3) << 17;
+  // per stage: Mp rows x 128 B of codes and row_tiles x 2 k-atoms of scales, per term
+  p.act_bytes = (static_cast<uint32_t>(Mp) * kBKBytes + row_tiles * 1024u) * (residual ? 2u : 1u);
+  p.skip_fill = skip_fill;
+  const int tiles = static_cast<int>((N + kBN - 1) / kBN);
+  if (residual)
+    return y_bf16 ? launch_typed<256, true, true, true>(maps, p, tiles, num_sms, stream)
+                  : launch_typed<256, true, false, true>(maps, p, tiles, num_sms, stream);
+  return y_bf16 ? launch_typed<256, false, true, true>(maps, p, tiles, num_sms, stream)
+                : launch_typed<256, false, false, true>(maps, p, tiles, num_sms, stream);
 }
 
 void set_fused_split_override(int split) { g_split_override.store(split < 0 ? 0 : split); }

@@ -123,6 +123,10 @@ rfq_status_t rfq_quantize_weight(const void* w_bf16, int64_t N, int64_t K,
  *   y            [M][N], y_type fp32 or bf16 (round to nearest even), 16-byte aligned
  * K multiple of 32; N multiple of 8.  M == 0 or N == 0 launches nothing;
  * K == 0 writes zeros.  Tensor cores: tcgen05 kind::mxf4 block-scaled MMAs.
+ * Short batches (M <= 256) whose output tiles would occupy less than half the
+ * SMs run a split-K kernel instead: 128 weight rows per CTA, K split over a
+ * cluster of up to 8 CTAs, partial sums added in a fixed order (the result
+ * differs from the tiled kernel's only by fp32 summation order).
  */
 rfq_status_t rfq_gemm(const void* qx_codes, const void* qx_scales,
                       const void* qr_codes, const void* qr_scales,
@@ -166,8 +170,8 @@ size_t rfq_linear_workspace_bytes(int64_t M, int64_t K, int use_residual);
  * rfq_linear -- the RFQ linear layer: rfq_quantize_mxfp4 of X into the caller's
  * workspace, then rfq_gemm against the pre-quantized weight, on one stream
  * (the method leaves the network unchanged: a drop-in for the layer's GEMM).
- * For 1 <= M <= RFQ_FUSED_MAX_M it runs rfq_linear_fused instead (same
- * arguments checked; the workspace is then left untouched).
+ * For 1 <= M <= 32 it runs rfq_linear_fused instead (same arguments checked;
+ * the workspace is then left untouched).
  *
  *   x_bf16          [M][K] bf16
  *   qw_codes/scales the weight as written by rfq_quantize_weight for [N][K]
@@ -219,7 +223,7 @@ rfq_status_t rfq_linear_wgrad(const void* x_bf16, const void* dy_bf16, int64_t M
                               void* workspace, size_t workspace_bytes,
                               cudaStream_t stream);
 
-/* Largest M that rfq_linear_fused accepts; rfq_linear uses it for 1 <= M <= this. */
+/* Largest M that rfq_linear_fused accepts (rfq_linear uses it for 1 <= M <= 32). */
 #define RFQ_FUSED_MAX_M 64
 
 /*

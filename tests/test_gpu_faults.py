@@ -8,7 +8,9 @@ also leave the producer waiting for a free stage, and either wait may expire fir
 records the wait in the device error word, drains its own copies and MMAs, frees its
 TMEM and returns; rfq_check_device_error reports RFQ_ERR_TIMEOUT with detail 1 (the
 stage wait) and the context stays usable: the next GEMM is correct.  Both the
-single-CTA path (M <= 128) and the CTA-pair path (M > 128) are exercised.
+single-CTA path (M <= 128 with enough columns to fill the GPU), the CTA-pair
+path (M > 256) and the short-batch split-K path (few tiles; K unsplit here so
+that the skipped fill is again the CTA's last) are exercised.
 """
 import numpy as np
 import pytest
@@ -19,10 +21,10 @@ from helpers import assert_y_close, dev_bf16, y_to_numpy
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("M", [128, 384])
-def test_skipped_fill_times_out_and_context_survives(rfq, oracle, M):
+@pytest.mark.parametrize("M,N", [(128, 256), (384, 256), (100, 19200)])
+def test_skipped_fill_times_out_and_context_survives(rfq, oracle, M, N):
     import torch
-    N, K = 256, 1024
+    K = 1024
     x_bits = wl.random_matrix(M, K, seed=M, scale=2.0)
     w_bits = wl.random_matrix(N, K, seed=M + 1, scale=0.05)
     qa = rfq.quantize_mxfp4_alloc(dev_bf16(x_bits), residual=True)
@@ -31,10 +33,14 @@ def test_skipped_fill_times_out_and_context_survives(rfq, oracle, M):
     rfq.check_device_error()
 
     rfq.debug_skip_next_fill(K // 256 - 1)   # the last of the tile's 256-K stage fills
+    rfq.debug_fused_split(1)
     y = torch.empty((M, N), dtype=torch.float32, device="cuda")
     rfq.gemm(qa.codes, qa.scales, qa.r_codes, qa.r_scales, qw.codes, qw.scales, M, N, K, y)
-    with pytest.raises(rfq.RFQError) as info:
-        rfq.check_device_error()
+    try:
+        with pytest.raises(rfq.RFQError) as info:
+            rfq.check_device_error()
+    finally:
+        rfq.debug_fused_split(0)
     assert info.value.status == 6          # RFQ_ERR_TIMEOUT
     assert info.value.detail == 1          # the MMA warp's wait for a loaded stage
     rfq.check_device_error()               # the error word was cleared

@@ -80,7 +80,7 @@ def test_fused_outlier_rows(rfq, oracle):
 
 
 def test_rfq_linear_dispatches_short_batches_to_fused(rfq):
-    """rfq_linear with M <= 64 runs the fused kernel: bit-identical to rfq_linear_fused
+    """rfq_linear with M <= 32 runs the fused kernel: bit-identical to rfq_linear_fused
     (same automatic split), and the workspace is left untouched."""
     import torch
     M, N, K = 32, 1024, 2048

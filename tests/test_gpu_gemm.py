@@ -59,8 +59,11 @@ def test_tiny_bf16_output(rfq, oracle):
     assert_y_close(y, Y, S, bf16_out=True)
 
 
+# Paths: M <= 256 with few tiles -> the short-batch split-K kernel; (100, 19200) the
+# single-CTA tiled GEMM (75 tiles); (200, 9472) and M > 256 the CTA-pair GEMM.
 @pytest.mark.parametrize("M,N,K", [(1, 8, 64), (16, 16, 64), (127, 136, 96), (129, 264, 160), (300, 520, 1024),
-                                   (256, 256, 4096), (64, 512, 32), (200, 1000, 2080)])
+                                   (256, 256, 4096), (64, 512, 32), (200, 1000, 2080), (100, 19200, 256),
+                                   (200, 9472, 288), (240, 4096, 1056)])
 @pytest.mark.parametrize("residual", [True, False])
 def test_edge_shapes(rfq, oracle, M, N, K, residual):
     import torch
@@ -143,3 +146,29 @@ def test_m_sweep_linear_sampled(rfq, oracle, M):
         Y, absY = oracle.gemm_blas(A, B)
         y = run_linear(rfq, wk.x_bits, wk.w_bits, residual, torch.bfloat16)
         assert_y_close(y[rows], Y, float(absY.max()), bf16_out=True, what=f"sweep M={M} res={residual}")
+
+
+@pytest.mark.parametrize("split", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("M", [40, 200])
+def test_short_batch_gemm_every_split(rfq, oracle, split, M):
+    """rfq_gemm on a short batch with few tiles runs the split-K kernel on the
+    quantizer's operands: each cluster size (9 k-tiles over 1..8 CTAs, ragged
+    ranges), one and two 128-row scale atoms of the activation, bit-identical
+    repeats."""
+    import torch
+    N, K = 384, 2304
+    x = wl.random_matrix(M, K, seed=M + split, scale=3.0)
+    w = wl.random_matrix(N, K, seed=17, scale=0.05)
+    Y, S, _ = oracle.rfq_linear(x, w, residual=True)
+    qa = rfq.quantize_mxfp4_alloc(dev_bf16(x))
+    qw = rfq.quantize_weight_alloc(dev_bf16(w))
+    rfq.debug_fused_split(split)
+    try:
+        ys = [rfq.gemm_alloc(qa, qw, out_dtype=out) for out in (torch.float32, torch.bfloat16, torch.float32)]
+        torch.cuda.synchronize()
+    finally:
+        rfq.debug_fused_split(0)
+    rfq.check_device_error()
+    assert_y_close(y_to_numpy(ys[0]), Y, S, bf16_out=False, what=f"short M={M} split {split}")
+    assert_y_close(y_to_numpy(ys[1]), Y, S, bf16_out=True, what=f"short M={M} split {split} bf16")
+    assert torch.equal(ys[0].view(torch.int32), ys[2].view(torch.int32))
