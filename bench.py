@@ -573,7 +573,7 @@ def run_cuda(args, rank, world, local):
         "gpu": torch.cuda.get_device_name(),
     }
     result.update(extra)
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:   # the CPU baseline is a 1-GPU figure
         result["cpu_baseline"] = cpu_baseline(wk, args.cpu_seconds)
     return result
 
