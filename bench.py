@@ -700,13 +700,25 @@ def run_single_kernel(args):
     rfq.load_library()
     M, K, N = args.M, args.K, args.N
     x = to_device_bf16(wl.random_matrix(M, K, seed=1, scale=2.0))
-    w = to_device_bf16(wl.random_matrix(N, K, seed=2, scale=0.05)) if args.kernel != "quantize" else x[:8]
+    w = to_device_bf16(wl.random_matrix(N, K, seed=2, scale=0.05)) if not args.kernel.startswith("quantize") \
+        else x[:8]
     step = RfqStep(rfq, x, w, residual=not args.no_rfq)
     step.quantize_w()
     step.quantize_x()
     fused = lambda: rfq.linear_fused(x, step.qw_c, step.qw_s, N, step.y, not args.no_rfq)
     fn = {"quantize": step.quantize_x, "gemm": step.gemm, "linear": step.run,
-          "two-kernel": lambda: (step.quantize_x(), step.gemm()), "fused": fused}[args.kernel]
+          "two-kernel": lambda: (step.quantize_x(), step.gemm()), "fused": fused}.get(args.kernel)
+    if args.kernel == "quantize-t":
+        # the operand of X^T (blocks along M), as for the weight-gradient GEMM
+        qt = rfq.quantize_mxfp4_t_alloc(x, residual=not args.no_rfq)
+        fn = lambda: rfq.quantize_mxfp4_t(x, qt.codes, qt.scales, qt.r_codes, qt.r_scales)
+    elif args.kernel == "gemm-yt":
+        yt = torch.empty((N, M), dtype=torch.bfloat16, device="cuda")
+        fn = lambda: rfq.gemm_yt(step.qx_c, step.qx_s, step.qr_c, step.qr_s, step.qw_c, step.qw_s, M, N, K, yt)
+    elif args.kernel in ("quantize-mxfp8", "gemm-mxfp8"):
+        q8a, q8w = rfq.quantize_mxfp8_alloc(x), rfq.quantize_mxfp8_alloc(w)
+        fn = (lambda: rfq.quantize_mxfp8(x, q8a.codes, q8a.scales)) if args.kernel == "quantize-mxfp8" else \
+            (lambda: rfq.gemm_mxfp8(q8a.codes, q8a.scales, q8w.codes, q8w.scales, M, N, K, step.y))
     rfq.debug_fused_split(args.split)
     t = time_kernel(fn, args.steps, make_l2_flush(torch))
     rfq.debug_fused_split(0)
@@ -715,8 +727,12 @@ def run_single_kernel(args):
     out = {"kernel": args.kernel, "M": M, "K": K, "N": N, "rfq": not args.no_rfq, "iters": args.steps,
            "split": args.split,
            "ms_mean": ms, "ms_min": min(t)}
-    if args.kernel == "quantize":
+    if args.kernel in ("quantize", "quantize-t"):
         out["gbs"] = quantize_bytes(M, K, not args.no_rfq) / (ms * 1e-3) / 1e9
+    elif args.kernel == "quantize-mxfp8":
+        out["gbs"] = (M * K * 3 + M * K // 32) / (ms * 1e-3) / 1e9
+    elif args.kernel == "gemm-mxfp8":
+        out["tflops"] = 2.0 * M * N * K / (ms * 1e-3) / 1e12
     else:
         out["tflops_executed"] = (2.0 if args.no_rfq else 4.0) * M * N * K / (ms * 1e-3) / 1e12
     print(json.dumps(out))
@@ -731,7 +747,8 @@ def main():
     ap.add_argument("--all-configs", action="store_true", help="also time the DiT FFN GEMM and the M sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
-    ap.add_argument("--kernel", choices=["quantize", "gemm", "linear", "two-kernel", "fused"], default=None,
+    ap.add_argument("--kernel", choices=["quantize", "gemm", "linear", "two-kernel", "fused", "quantize-t", "gemm-yt",
+                                         "quantize-mxfp8", "gemm-mxfp8"], default=None,
                     help="time one kernel on --M/--N/--K instead of the benchmark step (linear = quantize W "
                          "+ quantize X + GEMM; two-kernel = quantize X + GEMM; fused = rfq_linear_fused)")
     ap.add_argument("--split", type=int, default=0, help="with --kernel fused: K split (0 = automatic)")
