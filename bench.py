@@ -34,7 +34,7 @@ FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense MXFP4 : bf16 tensor throughp
 # profiles/rfq_quantize_kernel_M16384_K4096.md; the quantizer capture covers twice the
 # bench workload's units and is scaled by 1/2).  None once a kernel changes.
 NCU_TRAFFIC_BYTES = {"gemm_ffn_rfq_bf16": 46.314496e6 + 51.919872e6,
-                     "quantize_8192x4096_rfq": (134.412032e6 + 36.719104e6) / 2}
+                     "quantize_8192x4096_rfq": (134.372096e6 + 35.65056e6) / 2}
 L2_FLUSH_BYTES = 256 << 20
 
 

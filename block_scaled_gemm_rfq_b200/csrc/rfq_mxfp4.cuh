@@ -7,7 +7,7 @@
 // scale and E2M1 codes (OCP MX v1.0, section 6.3: scale exponent
 // floor(log2 amax) - emax_elem, emax_elem = 2 for E2M1; elements X / scale rounded
 // to nearest even, saturating to +-6); the residual R = X - DQ(Q(X)) is formed
-// exactly (in bf16 pairs, see quantize_block) and quantized by the same rule.
+// exactly (in fp32, see quantize_block) and quantized by the same rule.
 #pragma once
 
 #include <cstdint>
@@ -52,29 +52,41 @@ __device__ __forceinline__ void unpack_bf16x2(uint32_t w, float& lo, float& hi) 
   hi = __uint_as_float(w & 0xffff0000u);
 }
 
-// One word of 8 E2M1 codes -> their exact values as 4 bf16 pairs (element 2j in
-// the low half of word j).  The magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} are bf16
-// 0x0000, 0x3F00, 0x3F80, 0x3FC0, 0x4000, 0x4040, 0x4080, 0x40C0: two 8-entry
-// byte tables (high and low bytes) indexed by the 3 magnitude bits of 4 codes at
-// a time through byte permutes, then interleaved into pairs.  The sign of a code
-// is the sign of the element it was encoded from, so it is copied from the input
-// pair `xw[j]` (bf16 sign bits 15 and 31) instead of being decoded.
-__device__ __forceinline__ void decode8(uint32_t cw, const uint32_t* xw, uint32_t* out) {
-  const uint32_t mags = cw & 0x77777777u;
-  const uint32_t sel_lo = mags & 0xffffu, sel_hi = mags >> 16;
-  const uint32_t hi0 = prmt(0x3F3F3F00u, 0x40404040u, sel_lo), lo0 = prmt(0xC0800000u, 0xC0804000u, sel_lo);
-  const uint32_t hi1 = prmt(0x3F3F3F00u, 0x40404040u, sel_hi), lo1 = prmt(0xC0800000u, 0xC0804000u, sel_hi);
-  out[0] = prmt(lo0, hi0, 0x5140u) | (xw[0] & 0x80008000u);
-  out[1] = prmt(lo0, hi0, 0x7362u) | (xw[1] & 0x80008000u);
-  out[2] = prmt(lo1, hi1, 0x5140u) | (xw[2] & 0x80008000u);
-  out[3] = prmt(lo1, hi1, 0x7362u) | (xw[3] & 0x80008000u);
+// a * b + c on fp32 pairs (b shared by both), one rounding each.
+__device__ __forceinline__ void fma2(float& o0, float& o1, float a0, float a1, float b, float c0, float c1) {
+  asm("{\n\t.reg .b64 p, q, c, r;\n\t"
+      "mov.b64 p, {%2, %3};\n\t"
+      "mov.b64 q, {%4, %4};\n\t"
+      "mov.b64 c, {%5, %6};\n\t"
+      "fma.rn.f32x2 r, p, q, c;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(o0), "=f"(o1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c0), "f"(c1));
 }
 
-// a * b + c on bf16 pairs with one rounding (exact when the result is a bf16 value).
-__device__ __forceinline__ uint32_t bfma2(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
+// encode8, also returning the grid values the codes stand for (signed, exact) as
+// fp32: each code byte is decoded back by the hardware E2M1x2 -> f16x2
+// conversion (element 2j in the low half) and widened to fp32.
+__device__ __forceinline__ uint32_t encode8_dq(const float* v, float* q) {
+  uint32_t out, h[4];
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %8, %7;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %10, %9;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %12, %11;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %4, b3;\n\t}"
+      : "=r"(out), "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    asm("{\n\t.reg .f16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+        : "=f"(q[2 * j]), "=f"(q[2 * j + 1])
+        : "r"(h[j]));
+  return out;
 }
 
 // Per half: max(|a|, |b|) (with the XOR of the signs as sign, cleared by the
@@ -112,12 +124,15 @@ __device__ __forceinline__ float inv_scale(uint32_t s) { return __uint_as_float(
 // and byte of Q(R), R = X - DQ(Q(X)).  A non-finite block gets scale byte 0xFF
 // for both terms (its codes are unspecified).
 //
-// R is formed in bf16 pairs, exactly: with x an element (exponent e, so a
-// multiple of its bf16 ulp 2^(e-7)) and s the block's scale exponent (s >=
-// e - 2), DQ(Q(x)) is a multiple of 2^(s-1), hence of ulp(x), and the nearest
-// grid point is no farther from x than 0 is, so |x - DQ| <= |x|.  x - DQ is thus
-// a multiple of ulp(x) below 2^(e+1): a bf16 value, which one bf16 FMA returns
-// unrounded (saturated elements, |x| < 8 * 2^s against 6 * 2^s, too).
+// R is formed in fp32, exactly: with x an element (exponent e, so a multiple of
+// its bf16 ulp 2^(e-7)) and s the block's scale exponent (s >= e - 2), DQ(Q(x)) =
+// q * 2^s is a multiple of 2^(s-1), hence of ulp(x), and the nearest grid point
+// is no farther from x than 0 is, so |x - DQ| <= |x|.  x - DQ is thus a multiple
+// of ulp(x) below 2^(e+1), a bf16 (so also fp32) value; q * 2^s is exact too (q
+// has 2 significant bits, 2^-127 is an fp32 subnormal), so one fp32 FMA
+// q * (-2^s) + x returns R unrounded (saturated elements, |x| < 8 * 2^s against
+// 6 * 2^s, too).  R's elements being bf16 values, its amax has the exponent field
+// the bf16 rule reads.
 template <bool kResidual>
 __device__ __forceinline__ void quantize_block(const uint32_t (&w)[16], uint32_t (&cx)[4], uint32_t& sx_out,
                                                uint32_t (&cr)[4], uint32_t& sr_out) {
@@ -125,46 +140,49 @@ __device__ __forceinline__ void quantize_block(const uint32_t (&w)[16], uint32_t
   const uint32_t sx = scale_byte(block_amax_bits(w) >> 7);
   const uint32_t sx_eff = sx == 0xFFu ? 127u : sx;   // codes of a non-finite block are unspecified
   const float inv_x = inv_scale(sx_eff);
-  // -2^(sx-127) as a bf16 pair (byte 0: -2^-127, a bf16 subnormal)
-  const uint32_t neg_sc = sx_eff == 0u ? 0x8040u : (0x8000u | (sx_eff << 7));
-  const uint32_t neg_sc2 = neg_sc | (neg_sc << 16);
+  const float neg_sc = -__uint_as_float(sx_eff == 0u ? 0x00400000u : sx_eff << 23);   // -2^(sx-127)
 
-  // Per group of 8 elements: unpack bf16 -> fp32, scale (exact), encode; then
-  // decode and form the residual pairs.
-  uint32_t r2[16];
+  // Per group of 8 elements: unpack bf16 -> fp32, scale (exact), encode; with
+  // the residual, decode the codes and form R = x - q * 2^s.
+  float r[32];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    float v[8];
+    float x[8], v[8];
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      float x0, x1;
-      unpack_bf16x2(w[4 * k + h], x0, x1);
-      mul2(v[2 * h], v[2 * h + 1], x0, x1, inv_x);
+      unpack_bf16x2(w[4 * k + h], x[2 * h], x[2 * h + 1]);
+      mul2(v[2 * h], v[2 * h + 1], x[2 * h], x[2 * h + 1], inv_x);
     }
-    cx[k] = encode8(v);
     if constexpr (kResidual) {
-      uint32_t dq[4];
-      decode8(cx[k], w + 4 * k, dq);
+      float q[8];
+      cx[k] = encode8_dq(v, q);
 #pragma unroll
-      for (int h = 0; h < 4; ++h) r2[4 * k + h] = bfma2(dq[h], neg_sc2, w[4 * k + h]);
+      for (int h = 0; h < 4; ++h)
+        fma2(r[8 * k + 2 * h], r[8 * k + 2 * h + 1], q[2 * h], q[2 * h + 1], neg_sc, x[2 * h], x[2 * h + 1]);
+    } else {
+      cx[k] = encode8(v);
     }
   }
   sx_out = sx;
 
   if constexpr (kResidual) {
-    // ---- Q(R) by the same rule
-    uint32_t sr = scale_byte(block_amax_bits(r2) >> 7);
+    // ---- Q(R) by the same rule (R is finite when X is; a non-finite X block
+    // forces byte 0xFF)
+    float m[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m[i] = fmaxf(fabsf(r[2 * i]), fabsf(r[2 * i + 1]));
+#pragma unroll
+    for (int n = 8; n >= 1; n >>= 1)
+#pragma unroll
+      for (int i = 0; i < n; ++i) m[i] = fmaxf(m[i], m[i + n]);
+    uint32_t sr = scale_byte(__float_as_uint(m[0]) >> 23);
     if (sx == 0xFFu) sr = 0xFFu;
     const float inv_r = inv_scale(sr == 0xFFu ? 127u : sr);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       float v[8];
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        float r0, r1;
-        unpack_bf16x2(r2[4 * k + h], r0, r1);
-        mul2(v[2 * h], v[2 * h + 1], r0, r1, inv_r);
-      }
+      for (int h = 0; h < 4; ++h) mul2(v[2 * h], v[2 * h + 1], r[8 * k + 2 * h], r[8 * k + 2 * h + 1], inv_r);
       cr[k] = encode8(v);
     }
     sr_out = sr;

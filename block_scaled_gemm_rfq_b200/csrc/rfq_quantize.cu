@@ -7,7 +7,7 @@
 // it in one pass over X: every bf16 element is read from HBM exactly once and the
 // codes and E8M0 scales of Q(X) and Q(R) are written once, the scales directly in
 // the layout the block-scaled tensor-core MMA consumes.  R lives only in
-// registers, as bf16 pairs, in which it is exact (rfq_mxfp4.cuh).
+// registers, in fp32, in which it is exact (rfq_mxfp4.cuh).
 //
 // Work decomposition (HBM-bound streaming kernel, no tensor cores):
 //   * X is viewed as a flat sequence of 32-element blocks (64 bytes each; a block
@@ -17,9 +17,9 @@
 //   * every warp keeps kStages spans in flight with its own TMA ring (2-D tensor
 //     map over [blocks][64 bytes], 64-byte swizzle so that the lanes' 16-byte
 //     shared-memory reads are bank-conflict free) and mbarriers with bounded waits;
-//   * pairs of fp32 values go through packed f32x2 multiplies, the residual
-//     through bf16x2 FMAs and its amax through bf16x2 max, codes
-//     through cvt.rn.satfinite.e2m1x2.f32 (2 per instruction);
+//   * pairs of fp32 values go through packed f32x2 multiplies, codes through
+//     cvt.rn.satfinite.e2m1x2.f32 (2 per instruction) and back through
+//     cvt.rn.f16x2.e2m1x2 for the residual, which packed f32x2 FMAs form;
 //   * scale bytes: when K is a multiple of 128 the 4 lanes holding blocks
 //     4j..4j+3 of a row gather them into one 32-bit word of the MMA layout;
 //     otherwise each lane stores its byte.  The padding bytes of the scale
