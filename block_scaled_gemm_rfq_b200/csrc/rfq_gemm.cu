@@ -195,6 +195,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
+      if (unit < p.num_tiles) {
+        // While the previous kernel on the stream finishes, pull the first stages of
+        // this CTA's first tile into L2 (a hint; the copies still follow the wait).
+        const int mb = unit / p.num_nb, nb = unit - (unit / p.num_nb) * p.num_nb;
+        const int row_a = (mb * kPair + static_cast<int>(rank)) * kBM;
+        const int row_b = nb * kBN + static_cast<int>(rank) * (kBN / kPair);
+        for (int kt = 0; kt < L::kStages && kt < p.num_kt; ++kt) {
+          if (row_b < p.N) tma_prefetch_2d(&maps.w, kt * kBKBytes, row_b);
+          if (row_a < p.M) {
+            tma_prefetch_2d(&maps.x, kt * kBKBytes, row_a);
+            if (kResidual) tma_prefetch_2d(&maps.r, kt * kBKBytes, row_a);
+          }
+        }
+      }
       griddep_wait();   // QX/QR/QW may be written by the previous kernel on the stream
       uint32_t stage = 0, phase = 0;
       uint32_t filled = 0, last_parity = 0;

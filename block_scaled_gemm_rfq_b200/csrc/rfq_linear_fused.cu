@@ -225,6 +225,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     prefetch_tmap(&maps.w);
     prefetch_tmap(&maps.sw);
+    // With pre-quantized operands (after the quantizer on the stream), pull this CTA's
+    // slice of the weight into L2 while the previous kernel finishes (a hint; the
+    // copies still follow griddepcontrol.wait).  The bf16-input mode, which follows
+    // another short layer, measured slower with it.
+    if constexpr (kPreQ)
+      for (int i = 0; i < nk; ++i) tma_prefetch_2d(&maps.w, (kt0 + i) * kBKBytes, n0);
     griddep_wait();   // X and QW may be written by the previous kernel on the stream
     for (; issued < nk && issued < kStages; ++issued) issue_stage(issued);   // the stages start free
   }

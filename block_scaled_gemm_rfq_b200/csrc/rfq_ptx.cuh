@@ -113,6 +113,15 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                : "memory");
 }
 
+// Warm L2 with a tile of a tensor map (a hint: no data is returned, nothing waits
+// on it).  L2 is the point of coherence for device memory, so a tile prefetched
+// before griddepcontrol.wait returns cannot hide later writes of the previous
+// kernel from the loads issued after it.
+__device__ __forceinline__ void tma_prefetch_2d(const void* tmap, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(tmap), "r"(x), "r"(y)
+               : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }

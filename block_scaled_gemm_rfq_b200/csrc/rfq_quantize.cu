@@ -147,6 +147,9 @@ __global__ void __launch_bounds__(kThreads, RFQ_Q_CTAS_PER_SM)
   if (lane == 0) {
     for (int st = 0; st < kStages; ++st) mbar_init(&bars[st], 1);
     fence_mbar_init();
+    // While the previous kernel on the stream finishes, pull this warp's first
+    // spans into L2 (a hint; the copies below still follow griddepcontrol.wait).
+    for (uint32_t st = 0; st < kStages && st < n_my; ++st) tma_prefetch_2d(&tm_x, 0, span_row(gw + st * GW));
     griddep_wait();   // X may be written by the previous kernel on the stream
     for (uint32_t st = 0; st < kStages && st < n_my; ++st) {
       mbar_arrive_expect_tx(&bars[st], kSpanBytes);
