@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = unit; tile < p.num_tiles; tile += num_units) {
       const int mb = tile / p.num_nb;
       const int nb = tile - mb * p.num_nb;
-      if (!mbar_wait(acc_full, acc_phase, abort_flag, &g_device_error, kErrWaitAccFull)) break;
+      if (!mbar_wait(acc_full, acc_phase, abort_flag, &g_device_error, kErrWaitAccFull, 2 * kWaitLimitNs)) break;
       tc_fence_after();
       uint32_t v[4][32];
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + kAccCol + half * 128;

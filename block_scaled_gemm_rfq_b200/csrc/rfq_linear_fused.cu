@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the two warps of a lane quadrant alternate over 8-column chunks (rows of X).
     // With a K split the accumulator goes, as [Mp][128] fp32, to this CTA's
     // receive area for the cluster reduction below.
-    epi_ok = mbar_wait(acc_full, 0, abort_flag, &g_fused_error, kErrWaitAccFull);
+    epi_ok = mbar_wait(acc_full, 0, abort_flag, &g_fused_error, kErrWaitAccFull, 2 * kWaitLimitNs);
     if (__all_sync(0xffffffffu, epi_ok)) {
       tc_fence_after();
       const int quad = warp & 3;

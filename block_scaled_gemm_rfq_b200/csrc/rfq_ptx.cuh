@@ -68,10 +68,13 @@ __device__ __forceinline__ bool mbar_test_parity(uint32_t bar, uint32_t parity) 
 //
 // Wait until the phase with the given parity of `bar` has completed.  Bounded:
 // returns false (after recording `err` in *error_word and raising the
-// CTA's abort flag) when the wait runs past kWaitLimitNs, or as soon as another
-// role of the same CTA has raised the abort flag.
+// CTA's abort flag) when the wait runs past `limit_ns`, or as soon as another
+// role of the same CTA has raised the abort flag.  A wait that sits further down
+// the pipeline (the epilogue's, for the accumulator) passes twice the limit, so
+// that a stalled stage is reported by the wait nearest to it, which expires first.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned int* error_word, unsigned int err) {
+                                          unsigned int* error_word, unsigned int err,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_addr(bar);
   if (mbar_test_parity(a, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
@@ -80,7 +83,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     for (int i = 0; i < 64; ++i)
       if (mbar_test_parity(a, parity)) return true;
     if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       atomicCAS(error_word, 0u, err);
       *abort_flag = 1;
       return false;

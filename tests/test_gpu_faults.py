@@ -4,7 +4,8 @@ The library's test hook makes the producer of the first CTA skip one stage fill,
 the MMA warp's wait for that stage runs out (after about 1.5 s).  The skipped fill
 is the last one of the CTA's only tile: the producer then has nothing left to wait
 for, so the MMA warp's wait is the one that runs out (skipping an early fill would
-also leave the producer waiting for a free stage, and either wait may expire first).  The kernel then
+also leave the producer waiting for a free stage, and either wait may expire first;
+the epilogue's wait for the accumulator, which starts earlier, has twice the limit).  The kernel then
 records the wait in the device error word, drains its own copies and MMAs, frees its
 TMEM and returns; rfq_check_device_error reports RFQ_ERR_TIMEOUT with detail 1 (the
 stage wait) and the context stays usable: the next GEMM is correct.  Both the

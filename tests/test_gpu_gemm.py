@@ -74,6 +74,21 @@ def test_edge_shapes(rfq, oracle, M, N, K, residual):
     assert_y_close(y, Y, S, bf16_out=False, what=f"Y[{M}x{N}x{K}]")
 
 
+@pytest.mark.parametrize("M,N,K", [(2000, 2456, 256), (2048, 2560, 512), (4096, 4096, 256), (1800, 2696, 288)])
+@pytest.mark.parametrize("residual", [True, False])
+def test_partial_last_wave(rfq, oracle, M, N, K, residual):
+    """Tile counts (80, 80, 256, 88 pair tiles on 74 pairs) that leave a partial last
+    wave of the persistent schedule, with ragged M and N in the last tiles (the last
+    shape's final tile holds 136 real columns)."""
+    import torch
+    x = wl.random_matrix(M, K, seed=M + K, scale=2.0)
+    w = wl.random_matrix(N, K, seed=N + 3 * K, scale=0.05)
+    Y, S, _ = oracle.rfq_linear(x, w, residual=residual)
+    for out in (torch.float32, torch.bfloat16):
+        y = run_gemm(rfq, x, w, residual, out)
+        assert_y_close(y, Y, S, bf16_out=(out == torch.bfloat16), what=f"Y[{M}x{N}x{K}] {out}")
+
+
 def test_outlier_heavy_inputs(rfq, oracle):
     """Large dynamic range inside a row: outlier channels x1000 and tiny channels."""
     import torch
