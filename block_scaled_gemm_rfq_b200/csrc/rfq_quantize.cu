@@ -33,6 +33,7 @@
 #include "rfq_internal.h"
 #include "rfq_mxfp4.cuh"
 #include "rfq_ptx.cuh"
+#include "rfq_tmap.h"
 
 namespace rfq {
 
@@ -256,120 +257,193 @@ __global__ void __launch_bounds__(kThreads, RFQ_Q_CTAS_PER_SM)
 // ---------------------------------------------------------------- transposed quantizer
 // Quantizes X^T for a row-major bf16 X [R][C]: operand row c of the output is
 // column c of X, and its 32-element blocks run down 32 consecutive rows of X.
-// A warp takes units of 32 rows x 64 columns (4 KiB, one TMA box, kTStages in
-// flight); lane l reads, for each of the 32 rows, the 32-bit word holding columns
-// 2l and 2l+1 (conflict-free: a row's 32 words), regroups the halves into the
-// pair layout of a block (byte permutes) and quantizes the two columns' blocks
-// with the same per-block arithmetic as the row quantizer.  Units are ordered
-// row-block fastest, so warps running at the same time write neighbouring 16-byte
-// pieces of the same output rows.
+//
+// A CTA takes units of 256 rows x 64 columns of X: its 8 warps one 32-row block
+// each (a 4 KiB TMA box, kTStages in flight per warp).  Lane l reads, for each of
+// the 32 rows, the 32-bit word holding columns 2l and 2l+1 (conflict-free: a
+// row's 32 words), regroups the halves into the pair layout of a block (byte
+// permutes) and quantizes the two columns' blocks with the same per-block
+// arithmetic as the row quantizer.  The codes are not stored from the lanes
+// (16 bytes to each of 32 rows per store): the warps write them into a
+// shared-memory tile of 64 operand rows x 8 blocks (128-byte swizzle), and after
+// a CTA barrier one thread stores the tile with a TMA tensor store, so each
+// operand row receives 128 contiguous bytes; the scale bytes leave as 32-bit
+// words of the MMA layout.  The tiles are double-buffered: the store of one unit
+// overlaps the quantization of the next.  Units are ordered row-block fastest,
+// so CTAs running at the same time fill neighbouring pieces of the same rows.
 constexpr int kTWarps = 8;
 constexpr int kTThreads = kTWarps * 32;
-constexpr int kTStages = 3;
-constexpr uint32_t kTUnitBytes = 32 * 128;
-constexpr uint32_t kTSmemBytes = kTWarps * kTStages * kTUnitBytes + kTWarps * kTStages * 8 + 1024;
+constexpr int kTStages = 2;
+constexpr uint32_t kTUnitBytes = 32 * 128;           // one warp's box: 32 rows x 64 bf16
+constexpr uint32_t kTTileBytes = 64 * 128;           // codes of a unit: 64 operand rows x 8 blocks x 16 B
+constexpr uint32_t kTSfBytes = 64 * 8;               // scale bytes of a unit: 64 rows x 8 blocks
+constexpr uint32_t kTOffTileX = kTWarps * kTStages * kTUnitBytes;
+constexpr uint32_t kTOffTileR = kTOffTileX + 2 * kTTileBytes;
+constexpr uint32_t kTOffSfX = kTOffTileR + 2 * kTTileBytes;
+constexpr uint32_t kTOffSfR = kTOffSfX + 2 * kTSfBytes;
+constexpr uint32_t kTOffBars = kTOffSfR + 2 * kTSfBytes;
+constexpr uint32_t kTSmemBytes = kTOffBars + kTWarps * kTStages * 8 + 1024;
+static_assert(kTOffTileX % 1024 == 0 && kTOffTileR % 1024 == 0, "swizzled tiles need 1 KiB alignment");
 
 struct QuantTParams {
-  uint8_t* qt_codes;
   uint8_t* qt_scales;
-  uint8_t* qr_codes;
   uint8_t* qr_scales;
   uint32_t R;             // rows of X = K of the operand
   uint32_t C;             // columns of X = rows of the operand
   uint32_t Rb;            // R / 32: blocks per operand row
+  uint32_t Rb8;           // ceil(Rb / 8): units along R
   uint32_t kb4_per_tile;  // ceil(Rb / 4)
   uint32_t rows_pad;      // ceil(C / 128) * 128
   uint32_t num_ct;        // ceil(C / 64)
-  uint32_t num_units;     // Rb * num_ct
+  uint32_t num_units;     // Rb8 * num_ct
+};
+
+struct QuantTMaps {
+  CUtensorMap x;          // X [R][C] bf16, box 64 columns x 32 rows
+  CUtensorMap qt, qr;     // codes [C][R/2] bytes, box 128 B x 64 rows, 128-byte swizzle
 };
 
 template <bool kResidual>
 __global__ void __launch_bounds__(kTThreads, 2)
-    rfq_quantize_t_kernel(const __grid_constant__ CUtensorMap tm_x, const QuantTParams p) {
+    rfq_quantize_t_kernel(const __grid_constant__ QuantTMaps maps, const QuantTParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   uint8_t* ring = smem + warp * (kTStages * kTUnitBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTWarps * kTStages * kTUnitBytes) + warp * kTStages;
-  volatile int abort_flag = 0;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTOffBars) + warp * kTStages;
+  volatile int abort_flag = 0;   // per warp: each warp's ring is independent
 
-  const uint32_t gw = blockIdx.x * kTWarps + warp;
-  const uint32_t GW = gridDim.x * kTWarps;
-  const uint32_t n_my = p.num_units > gw ? (p.num_units - gw + GW - 1) / GW : 0;
+  const uint32_t n_my =
+      p.num_units > blockIdx.x ? (p.num_units - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;   // CTA-uniform
+  // Block row rt of X this warp quantizes in the CTA's k-th unit, and its column tile.
+  auto unit_of = [&](uint32_t k, uint32_t& rt, uint32_t& ct) {
+    const uint32_t u = blockIdx.x + k * gridDim.x;
+    ct = u / p.Rb8;
+    rt = (u - ct * p.Rb8) * kTWarps + static_cast<uint32_t>(warp);
+  };
   auto issue = [&](uint32_t k, int st) {
-    const uint32_t u = gw + k * GW;
-    const uint32_t rt = u % p.Rb, ct = u / p.Rb;
-    mbar_arrive_expect_tx(&bars[st], kTUnitBytes);
-    tma_load_2d(ring + st * kTUnitBytes, &tm_x, &bars[st], static_cast<int>(ct * 64), static_cast<int>(rt * 32));
+    uint32_t rt, ct;
+    unit_of(k, rt, ct);
+    if (rt < p.Rb) {
+      mbar_arrive_expect_tx(&bars[st], kTUnitBytes);
+      tma_load_2d(ring + st * kTUnitBytes, &maps.x, &bars[st], static_cast<int>(ct * 64), static_cast<int>(rt * 32));
+    } else {
+      mbar_arrive(&bars[st]);   // past the last block row: nothing to load, the phase still completes
+    }
   };
 
   griddep_launch_dependents();
   if (lane == 0) {
     for (int st = 0; st < kTStages; ++st) mbar_init(&bars[st], 1);
     fence_mbar_init();
+    if (warp == 0) {
+      prefetch_tmap(&maps.qt);
+      if (kResidual) prefetch_tmap(&maps.qr);
+    }
+    // While the previous kernel on the stream finishes, pull this warp's first boxes
+    // into L2 (a hint; the copies below still follow griddepcontrol.wait).
+    for (uint32_t k = 0; k < kTStages && k < n_my; ++k) {
+      uint32_t rt, ct;
+      unit_of(k, rt, ct);
+      if (rt < p.Rb) tma_prefetch_2d(&maps.x, static_cast<int>(ct * 64), static_cast<int>(rt * 32));
+    }
     griddep_wait();   // X may be written by the previous kernel on the stream
     for (uint32_t k = 0; k < kTStages && k < n_my; ++k) issue(k, static_cast<int>(k));
   }
   __syncwarp();
 
-  uint32_t i = 0;
-  for (; i < n_my; ++i) {
-    const int st = static_cast<int>(i % kTStages);
-    const bool ok = mbar_wait(&bars[st], (i / kTStages) & 1u, &abort_flag, &g_quant_error, kErrQuantWait);
-    if (!__all_sync(0xffffffffu, ok)) break;
+  bool ok = true;            // this warp's waits so far (warp-uniform)
+  uint32_t k_fail = n_my;    // the unit whose wait ran out
+  uint32_t k = 0;
+  for (; k < n_my; ++k) {
+    const int st = static_cast<int>(k % kTStages);
+    const uint32_t buf = k & 1u;
+    uint32_t rt, ct;
+    unit_of(k, rt, ct);
+    uint8_t* tile_x = smem + kTOffTileX + buf * kTTileBytes;
+    uint8_t* tile_r = smem + kTOffTileR + buf * kTTileBytes;
+    uint8_t* sf_x = smem + kTOffSfX + buf * kTSfBytes;
+    uint8_t* sf_r = smem + kTOffSfR + buf * kTSfBytes;
+    // A wait that runs out leaves the warp producing garbage without waiting again:
+    // every warp still reaches each CTA barrier below, and the error word reports it.
+    if (ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[st], (k / kTStages) & 1u, &abort_flag, &g_quant_error,
+                                             kErrQuantWait));
+      if (!ok) k_fail = k;
+    }
     uint32_t wr[32];
     const uint32_t* src = reinterpret_cast<const uint32_t*>(ring + st * kTUnitBytes) + lane;
 #pragma unroll
     for (int r = 0; r < 32; ++r) wr[r] = src[r * 32];
     __syncwarp();
-    if (lane == 0 && i + kTStages < n_my) {
+    if (lane == 0 && ok && k + kTStages < n_my) {
+      // this warp's data are in registers: refill the stage (reads ordered before the async write)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue(i + kTStages, st);
+      issue(k + kTStages, st);
     }
-    const uint32_t u = gw + i * GW;
-    const uint32_t rt = u % p.Rb, ct = u / p.Rb;
+    const bool valid = rt < p.Rb;   // warp-uniform
 #pragma unroll 1
     for (int h = 0; h < 2; ++h) {
       // element 2j of the block = row 2j (low half), 2j+1 = row 2j+1 (high half)
       uint32_t w[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) w[j] = prmt(wr[2 * j], wr[2 * j + 1], h ? 0x7632u : 0x5410u);
-      uint32_t cx[4], cr[4], sx, sr;
-      quantize_block<kResidual>(w, cx, sx, cr, sr);
-      const uint32_t c = ct * 64 + 2 * lane + h;
-      if (c < p.C) {
-        const size_t code_off = static_cast<size_t>(c) * (p.R / 2) + rt * 16;
-        const uint32_t sf_off = scale_word_offset(c, rt >> 2, p.kb4_per_tile) + (rt & 3);
-        *reinterpret_cast<uint4*>(p.qt_codes + code_off) = make_uint4(cx[0], cx[1], cx[2], cx[3]);
-        p.qt_scales[sf_off] = static_cast<uint8_t>(sx);
-        if constexpr (kResidual) {
-          *reinterpret_cast<uint4*>(p.qr_codes + code_off) = make_uint4(cr[0], cr[1], cr[2], cr[3]);
-          p.qr_scales[sf_off] = static_cast<uint8_t>(sr);
-        }
+      uint32_t cx[4] = {0, 0, 0, 0}, cr[4] = {0, 0, 0, 0}, sx = 0, sr = 0;
+      if (valid) quantize_block<kResidual>(w, cx, sx, cr, sr);
+      // operand row 2 lane + h of the tile, block `warp`: 16-byte chunk `warp` of the
+      // row's 128 bytes, at chunk position warp ^ (row % 8) (128-byte swizzle)
+      const uint32_t r_loc = 2u * static_cast<uint32_t>(lane) + static_cast<uint32_t>(h);
+      const uint32_t off = r_loc * 128u + ((static_cast<uint32_t>(warp) ^ (r_loc & 7u)) << 4);
+      *reinterpret_cast<uint4*>(tile_x + off) = make_uint4(cx[0], cx[1], cx[2], cx[3]);
+      sf_x[r_loc * 8u + warp] = static_cast<uint8_t>(sx);   // 0 past the last block row: scale padding
+      if constexpr (kResidual) {
+        *reinterpret_cast<uint4*>(tile_r + off) = make_uint4(cr[0], cr[1], cr[2], cr[3]);
+        sf_r[r_loc * 8u + warp] = static_cast<uint8_t>(sr);
+      }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the tiles go out through TMA
+    // The other buffer's store (issued one unit ago) must have finished reading it
+    // before the barrier lets the warps write it again in the next unit.
+    if (threadIdx.x == 0) bulk_wait_read_all();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const int x = static_cast<int>((rt - static_cast<uint32_t>(warp)) * 16u), y = static_cast<int>(ct * 64u);
+      tma_store_2d(&maps.qt, tile_x, x, y);
+      if (kResidual) tma_store_2d(&maps.qr, tile_r, x, y);
+      bulk_commit_group();
+    }
+    if (threadIdx.x < 128) {
+      // scales: operand row c, 4-block word j of the unit's 8 blocks
+      const uint32_t r_loc = threadIdx.x >> 1, j = threadIdx.x & 1u;
+      const uint32_t c = ct * 64u + r_loc;
+      const uint32_t kb4 = (rt - static_cast<uint32_t>(warp)) / 4u + j;   // rt - warp: the unit's first block row
+      if (c < p.C && kb4 < p.kb4_per_tile) {
+        const uint32_t o = scale_word_offset(c, kb4, p.kb4_per_tile);
+        *reinterpret_cast<uint32_t*>(p.qt_scales + o) = *reinterpret_cast<const uint32_t*>(sf_x + r_loc * 8u + 4u * j);
+        if constexpr (kResidual)
+          *reinterpret_cast<uint32_t*>(p.qr_scales + o) = *reinterpret_cast<const uint32_t*>(sf_r + r_loc * 8u + 4u * j);
       }
     }
   }
 
-  if (i < n_my && lane == 0) {
-    // A wait ran out: let this warp's outstanding copies land before leaving.
+  if (!ok && lane == 0) {
+    // A wait ran out: let this warp's outstanding copies (units k_fail .. k_fail +
+    // kTStages - 1, issued before it) land before leaving.
     int never = 0;
-    for (uint32_t k = i; k < n_my && k < i + kTStages; ++k)
-      mbar_wait(&bars[k % kTStages], static_cast<uint32_t>((k / kTStages) & 1), &never, &g_quant_error,
-                kErrQuantWait);
+    for (uint32_t i = k_fail; i < n_my && i < k_fail + kTStages; ++i)
+      mbar_wait(&bars[i % kTStages], (i / kTStages) & 1u, &never, &g_quant_error, kErrQuantWait);
   }
+  if (threadIdx.x == 0) bulk_wait_all();   // the tiles' stores are complete before the CTA's memory goes
 
   griddep_wait();   // the padding stores may hit buffers the previous kernel still reads
   zero_scale_padding(p.qt_scales, kResidual ? p.qr_scales : nullptr, p.C, p.Rb, p.kb4_per_tile, p.rows_pad,
                      blockIdx.x * kTThreads + threadIdx.x, gridDim.x * kTThreads);
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 template <bool kResidual>
-cudaError_t launch_t_typed(const CUtensorMap& tm, const QuantTParams& p, int grid, cudaStream_t stream) {
+cudaError_t launch_t_typed(const QuantTMaps& maps, const QuantTParams& p, int grid, cudaStream_t stream) {
   auto kernel = rfq_quantize_t_kernel<kResidual>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTSmemBytes);
   if (e != cudaSuccess) return e;
@@ -383,7 +457,7 @@ cudaError_t launch_t_typed(const CUtensorMap& tm, const QuantTParams& p, int gri
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kernel, tm, p);
+  e = cudaLaunchKernelEx(&cfg, kernel, maps, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -478,36 +552,42 @@ cudaError_t launch_quantize_mxfp8(const void* x, int64_t M, int64_t K, void* cod
 cudaError_t launch_quantize_t(const void* x, int64_t R, int64_t C, void* qt_codes, void* qt_scales, void* qr_codes,
                               void* qr_scales, int num_sms, void* encode_tiled, cudaStream_t stream) {
   QuantTParams p;
-  p.qt_codes = static_cast<uint8_t*>(qt_codes);
   p.qt_scales = static_cast<uint8_t*>(qt_scales);
-  p.qr_codes = static_cast<uint8_t*>(qr_codes);
   p.qr_scales = static_cast<uint8_t*>(qr_scales);
   p.R = static_cast<uint32_t>(R);
   p.C = static_cast<uint32_t>(C);
   p.Rb = static_cast<uint32_t>(R / 32);
+  p.Rb8 = (p.Rb + kTWarps - 1) / kTWarps;
   p.kb4_per_tile = (p.Rb + 3) / 4;
   p.rows_pad = static_cast<uint32_t>((C + 127) / 128 * 128);
   p.num_ct = static_cast<uint32_t>((C + 63) / 64);
-  p.num_units = p.Rb * p.num_ct;
+  p.num_units = p.Rb8 * p.num_ct;
 
   // X as [R][C] 16-bit elements; boxes of 64 columns x 32 rows, no swizzle, zeros
-  // past the last column.
-  CUtensorMap tm;
+  // past the last column.  The codes as [C][R/2] bytes, stored in 128-byte x
+  // 64-row tiles (128-byte swizzle, clipped at the ends).
+  QuantTMaps maps;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(R)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(C) * 2};
   cuuint32_t box[2] = {64u, 32u};
   cuuint32_t elem_strides[2] = {1, 1};
   EncodeTiledFn encode = reinterpret_cast<EncodeTiledFn>(encode_tiled);
-  if (encode(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(x), dims, strides, box, elem_strides,
+  if (encode(&maps.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(x), dims, strides, box, elem_strides,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  int64_t grid = (static_cast<int64_t>(p.num_units) + kTWarps - 1) / kTWarps;
+  if (!encode_code_rows_map(encode, &maps.qt, qt_codes, C, R / 2, 64)) return cudaErrorInvalidValue;
+  if (qr_codes) {
+    if (!encode_code_rows_map(encode, &maps.qr, qr_codes, C, R / 2, 64)) return cudaErrorInvalidValue;
+  } else {
+    maps.qr = maps.qt;
+  }
+  int64_t grid = static_cast<int64_t>(p.num_units);
   const int64_t cap = static_cast<int64_t>(num_sms) * 2;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  return qr_codes ? launch_t_typed<true>(tm, p, static_cast<int>(grid), stream)
-                  : launch_t_typed<false>(tm, p, static_cast<int>(grid), stream);
+  return qr_codes ? launch_t_typed<true>(maps, p, static_cast<int>(grid), stream)
+                  : launch_t_typed<false>(maps, p, static_cast<int>(grid), stream);
 }
 
 cudaError_t read_and_clear_quant_error(unsigned int* value) {
