@@ -33,7 +33,7 @@ FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense MXFP4 : bf16 tensor throughp
 # kernels (profiles/rfq_gemm_kernel_pair_ffn_up_M4096_K4096_N12288.md and
 # profiles/rfq_quantize_kernel_M16384_K4096.md; the quantizer capture covers twice the
 # bench workload's units and is scaled by 1/2).  None once a kernel changes.
-NCU_TRAFFIC_BYTES = {"gemm_ffn_rfq_bf16": 46.8672e6 + 54.359552e6,
+NCU_TRAFFIC_BYTES = {"gemm_ffn_rfq_bf16": 47.675904e6 + 61.370368e6,
                      "quantize_8192x4096_rfq": (134.38208e6 + 37.032704e6) / 2}
 L2_FLUSH_BYTES = 256 << 20
 

@@ -66,7 +66,10 @@ constexpr uint32_t kSfaRCol = 8;       // +8+4a..:     QR
 constexpr uint32_t kSfbCol = 16;       // +16+8a..+7:  QW, the tile's 256 rows (2 row atoms)
 constexpr uint32_t kSmemLimit = 232448;
 
-template <int kPair>
+// kYTile: the epilogue stages Y in shared memory (8 warps x two 4 KiB boxes of 32
+// rows x 64 bf16, 128-byte swizzle) and stores it with TMA tensor stores; the
+// ring gives up a stage for it (3 stages measured as fast as 4).
+template <int kPair, bool kYTile = false>
 struct Layout {
   static constexpr uint32_t kATile = kBM * kBKBytes;                 // 16 KiB
   static constexpr uint32_t kBTile = (kBN / kPair) * kBKBytes;       // 32 KiB (single) or 16 KiB (pair)
@@ -78,9 +81,14 @@ struct Layout {
   static constexpr uint32_t kOffSfb = kOffSfaR + 1024;               // [row atom lo, hi][k-atom 0, 1]
   static constexpr uint32_t kStage = kOffSfb + 2048;
   static constexpr uint32_t kBarrierBytes = 256;
-  static constexpr int kStages = static_cast<int>((kSmemLimit - 1024 - kBarrierBytes) / kStage);
-  static constexpr uint32_t kSmem = kStages * kStage + kBarrierBytes + 1024;
+  static constexpr uint32_t kYBox = 32 * 128;                         // 32 rows x 64 bf16
+  static constexpr uint32_t kYBytes = kYTile ? 16 * kYBox : 0u;       // 8 epilogue warps x 2 boxes
+  static constexpr int kStages = static_cast<int>((kSmemLimit - 1024 - kBarrierBytes - kYBytes) / kStage);
+  static constexpr uint32_t kOffY = kStages * kStage;
+  static constexpr uint32_t kSmem = kStages * kStage + kYBytes + kBarrierBytes + 1024;
   static_assert(kStage % 1024 == 0, "stage buffers must keep 1 KiB alignment");
+  static_assert(kStages >= 3, "the ring needs at least 3 stages");
+  static_assert(kOffY % 1024 == 0, "the Y boxes need 1 KiB alignment (128-byte swizzle)");
   static_assert(kSmem <= kSmemLimit, "exceeds the 227 KiB shared-memory limit");
   static_assert((2 * kStages + 3) * 8 + 8 <= kBarrierBytes, "barrier area too small");
   static_assert(kSfBase + kStages * kSfSlot <= kTmemCols, "scale slots exceed TMEM");
@@ -99,6 +107,7 @@ struct GemmParams {
 struct Maps {
   CUtensorMap x, r, w;           // codes: [rows][K/2] bytes, box 128 B x (128 | 256 | 128) rows, 128-byte swizzle
   CUtensorMap sx, sr, sw;        // scales: [row tiles][k atoms][2][256 B]; box = 2 k-atoms of 1 (A) or 2 (B) row tiles
+  CUtensorMap y;                 // Y [M][N] bf16, box 64 columns x 32 rows, 128-byte swizzle (kYTile)
 };
 
 // Shared-memory matrix descriptor (tcgen05): K-major operand, 128-byte swizzle,
@@ -137,7 +146,8 @@ __device__ __forceinline__ uint32_t mma_idesc(uint32_t sf_id) {
 template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     rfq_gemm_kernel(const __grid_constant__ Maps maps, const GemmParams p) {
-  using L = Layout<kPair>;
+  constexpr bool kYTile = kBf16Out && !kTransOut && kPair == 2;
+  using L = Layout<kPair, kYTile>;
   // A stage is 128 bytes of codes per row either way: 256 K of FP4 (2 scale atoms
   // per operand row tile) or 128 K of FP8 (1 atom).
   constexpr int kKAtoms = kFp8 ? 1 : 2;
@@ -145,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kSfbBytes = 2u * 512u * kKAtoms;   // two row tiles (256 rows of W)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStage);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStage + L::kYBytes);
   uint64_t* empty = full + L::kStages;
   uint64_t* acc_full = empty + L::kStages;
   uint64_t* acc_empty = acc_full + 1;
@@ -363,7 +373,41 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       const int row = (mb * kPair + static_cast<int>(rank)) * kBM + quad * 32 + lane;
       const int col0 = nb * kBN + half * 128;
-      if constexpr (kTransOut) {
+      if constexpr (kYTile) {
+        // Y through shared memory and TMA: this warp's 32 rows x 128 columns as two
+        // boxes of 64 columns (128-byte rows; 16-byte chunk j of row r at position
+        // j ^ (r % 8), the 128-byte swizzle), so Y leaves in whole 128-byte row pieces
+        // instead of 16 bytes to each of 32 rows per warp store.
+        uint8_t* ybox = smem + L::kOffY + static_cast<uint32_t>(warp - 2) * 2u * L::kYBox;
+        if (lane == 0) bulk_wait_read_all();   // this warp's stores of the previous tile have read the boxes
+        __syncwarp();
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            uint32_t pw[4];
+#pragma unroll
+            for (int hh = 0; hh < 4; ++hh) {
+              const int e = 64 * cc + 8 * j + 2 * hh;
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[e >> 5][e & 31]),
+                                                        __uint_as_float(v[(e + 1) >> 5][(e + 1) & 31]));
+              pw[hh] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            *reinterpret_cast<uint4*>(ybox + cc * L::kYBox + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(pw[0], pw[1], pw[2], pw[3]);
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the boxes go out through TMA
+        __syncwarp();
+        if (lane == 0) {
+          const int y0 = row - lane;   // the warp's first row
+          if (y0 < p.M) {              // boxes past the end are not stored (nothing of them is in Y)
+            if (col0 < p.N) tma_store_2d(&maps.y, ybox, col0, y0);
+            if (col0 + 64 < p.N) tma_store_2d(&maps.y, ybox + L::kYBox, col0 + 64, y0);
+          }
+          bulk_commit_group();
+        }
+      } else if constexpr (kTransOut) {
         // Y^T [N][M]: for each column the warp's 32 lanes hold 32 consecutive rows,
         // so one store per column writes 32 neighbouring elements of a row of Y^T.
         if (row < p.M) {
@@ -406,6 +450,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if constexpr (kYTile) {
+      if (lane == 0) bulk_wait_all();   // Y's stores are complete before the CTA's memory goes
+    }
   }
 
   tc_fence_before();
@@ -421,12 +468,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut, bool kFp8 = false>
 cudaError_t launch_typed(const Maps& maps, const GemmParams& p, int grid, cudaStream_t stream) {
   auto kernel = rfq_gemm_kernel<kPair, kResidual, kBf16Out, kTransOut, kFp8>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<kPair>::kSmem);
+  using L = Layout<kPair, kBf16Out && !kTransOut && kPair == 2>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = Layout<kPair>::kSmem;
+  cfg.dynamicSmemBytes = L::kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -478,6 +526,19 @@ cudaError_t launch_gemm_impl(const void* qx_codes, const void* qx_scales, const 
     return cudaErrorInvalidValue;
   if (!encode_scales_map(encode, &maps.sx, qx_scales, M, K, 1, katoms)) return cudaErrorInvalidValue;
   if (!encode_scales_map(encode, &maps.sw, qw_scales, N, K, 2, katoms)) return cudaErrorInvalidValue;
+  if (pair && y_bf16 && !y_transposed) {
+    // Y [M][N] bf16 for the TMA-store epilogue: boxes of 64 columns x 32 rows
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {64u, 32u};
+    cuuint32_t elem_strides[2] = {1, 1};
+    if (encode(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, elem_strides,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    maps.y = maps.x;   // unused
+  }
   if (residual) {
     if (!encode_code_rows_map(encode, &maps.r, qr_codes, M, row_bytes, kBM)) return cudaErrorInvalidValue;
     if (!encode_scales_map(encode, &maps.sr, qr_scales, M, K, 1, katoms)) return cudaErrorInvalidValue;
