@@ -68,7 +68,12 @@ constexpr uint32_t kSmemLimit = 232448;
 
 // kYTile: the epilogue stages Y in shared memory (8 warps x two 4 KiB boxes of 32
 // rows x 64 bf16, 128-byte swizzle) and stores it with TMA tensor stores; the
-// ring gives up a stage for it (3 stages measured as fast as 4).
+// ring gives up a stage for it.  Only the RFQ kernel with CTA pairs and bf16 Y:
+// there 3 stages measured as fast as 4, while the kernels with half the MMAs per
+// stage (RFQ off, MXFP8) lost 10-13 % with 3.
+template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut, bool kFp8>
+constexpr bool kYTileFor = kPair == 2 && kResidual && kBf16Out && !kTransOut && !kFp8;
+
 template <int kPair, bool kYTile = false>
 struct Layout {
   static constexpr uint32_t kATile = kBM * kBKBytes;                 // 16 KiB
@@ -146,7 +151,7 @@ __device__ __forceinline__ uint32_t mma_idesc(uint32_t sf_id) {
 template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     rfq_gemm_kernel(const __grid_constant__ Maps maps, const GemmParams p) {
-  constexpr bool kYTile = kBf16Out && !kTransOut && kPair == 2;
+  constexpr bool kYTile = kYTileFor<kPair, kResidual, kBf16Out, kTransOut, kFp8>;
   using L = Layout<kPair, kYTile>;
   // A stage is 128 bytes of codes per row either way: 256 K of FP4 (2 scale atoms
   // per operand row tile) or 128 K of FP8 (1 atom).
@@ -468,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut, bool kFp8 = false>
 cudaError_t launch_typed(const Maps& maps, const GemmParams& p, int grid, cudaStream_t stream) {
   auto kernel = rfq_gemm_kernel<kPair, kResidual, kBf16Out, kTransOut, kFp8>;
-  using L = Layout<kPair, kBf16Out && !kTransOut && kPair == 2>;
+  using L = Layout<kPair, kYTileFor<kPair, kResidual, kBf16Out, kTransOut, kFp8>>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
