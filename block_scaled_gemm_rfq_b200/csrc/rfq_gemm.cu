@@ -28,8 +28,10 @@
 //               MMAs of K = 64; tcgen05.commit frees the stage and, at the end of
 //               a tile, signals the epilogues;
 //   warps 2..9  epilogue: TMEM -> registers (128 columns per warp), release of
-//               the accumulator, then fp32/bf16 -> global, one row per thread,
-//               overlapping the next tile's mainloop.
+//               the accumulator, then fp32/bf16 -> global, overlapping the next
+//               tile's mainloop: one row per thread, or (RFQ, pairs, bf16 Y)
+//               through swizzled shared-memory boxes and TMA tensor stores.
+// Before its dependency wait the producer prefetches its first stages into L2.
 // Every mbarrier wait is bounded (rfq_ptx.cuh); a wait that runs out records an
 // error code, raises the CTA's abort flag and the CTA tears down cleanly.  No TMA
 // multicast is used anywhere (the pair's loads each fill their own CTA).
