@@ -63,15 +63,19 @@ def test_tiny_bf16_output(rfq, oracle):
 # single-CTA tiled GEMM (75 tiles); (200, 9472) and M > 256 the CTA-pair GEMM.
 @pytest.mark.parametrize("M,N,K", [(1, 8, 64), (16, 16, 64), (127, 136, 96), (129, 264, 160), (300, 520, 1024),
                                    (256, 256, 4096), (64, 512, 32), (200, 1000, 2080), (100, 19200, 256),
-                                   (200, 9472, 288), (240, 4096, 1056)])
+                                   (200, 9472, 288), (240, 4096, 1056), (300, 8, 64), (333, 136, 128),
+                                   (1000, 72, 256)])
 @pytest.mark.parametrize("residual", [True, False])
 def test_edge_shapes(rfq, oracle, M, N, K, residual):
+    """fp32 and bf16 Y (bf16 with CTA pairs and the residual goes through the
+    TMA-store epilogue, whose boxes are clipped at ragged M and N)."""
     import torch
     x = wl.random_matrix(M, K, seed=M + 3 * N + 7 * K, scale=2.0)
     w = wl.random_matrix(N, K, seed=M * N + K, scale=0.05)
     Y, S, _ = oracle.rfq_linear(x, w, residual=residual)
-    y = run_gemm(rfq, x, w, residual, torch.float32)
-    assert_y_close(y, Y, S, bf16_out=False, what=f"Y[{M}x{N}x{K}]")
+    for out in (torch.float32, torch.bfloat16):
+        y = run_gemm(rfq, x, w, residual, out)
+        assert_y_close(y, Y, S, bf16_out=(out == torch.bfloat16), what=f"Y[{M}x{N}x{K}] {out}")
 
 
 @pytest.mark.parametrize("M,N,K", [(2000, 2456, 256), (2048, 2560, 512), (4096, 4096, 256), (1800, 2696, 288)])
