@@ -30,9 +30,9 @@ sys.path.insert(0, ROOT)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense MXFP4 : bf16 tensor throughput on B200
 # DRAM bytes (read + write) per launch from `ncu --set full` captures of the current
-# kernels (profiles/rfq_gemm_kernel_pair_ffn_up_M4096_K4096_N12288.md and
-# profiles/rfq_quantize_kernel_M16384_K4096.md; the quantizer capture covers twice the
-# bench workload's units and is scaled by 1/2).  None once a kernel changes.
+# kernels (the GEMM on this FFN workload; the quantizer on 16384 x 4096, twice the
+# bench workload's units, scaled by 1/2; summaries under profiles/).  None once a
+# kernel changes.
 NCU_TRAFFIC_BYTES = {"gemm_ffn_rfq_bf16": 47.675904e6 + 61.370368e6,
                      "quantize_8192x4096_rfq": (134.38208e6 + 37.032704e6) / 2}
 L2_FLUSH_BYTES = 256 << 20
