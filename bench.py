@@ -36,6 +36,7 @@ FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense MXFP4 : bf16 tensor throughp
 NCU_TRAFFIC_BYTES = {"gemm_ffn_rfq_bf16": 47.675904e6 + 61.370368e6,
                      "quantize_8192x4096_rfq": (134.38208e6 + 37.032704e6) / 2}
 L2_FLUSH_BYTES = 256 << 20
+REFERENCE_RUN_SECONDS = 150.0   # host time of a whole --impl reference run
 
 
 def make_l2_flush(torch):
@@ -620,11 +621,15 @@ def run_reference(args):
     samples, reported in the same metric/unit."""
     from block_scaled_gemm_rfq_b200 import workloads as wl
     wk = wl.ffn_up(seed=0)
+    # Each step's sample shrinks with the number of steps so that the whole run stays
+    # near REFERENCE_RUN_SECONDS of host time (the GEMM part of a sample is timed over
+    # a third of its budget; the quantizer rows are fixed, ~0.25 s).
+    budget = max(0.3, min(args.cpu_seconds, REFERENCE_RUN_SECONDS / max(1, args.steps + args.warmup)))
     samples = []
     for _ in range(args.warmup):
-        cpu_baseline(wk, args.cpu_seconds)
+        cpu_baseline(wk, budget)
     for _ in range(args.steps):
-        samples.append(cpu_baseline(wk, args.cpu_seconds))
+        samples.append(cpu_baseline(wk, budget))
     v = statistics.mean(s["value"] for s in samples)
     cb = dict(samples[-1])
     cb["value"] = v
