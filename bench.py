@@ -34,7 +34,7 @@ FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense MXFP4 : bf16 tensor throughp
 # bench workload's units, scaled by 1/2; summaries under profiles/).  None once a
 # kernel changes.
 NCU_TRAFFIC_BYTES = {"gemm_ffn_rfq_bf16": 47.675904e6 + 61.370368e6,
-                     "quantize_8192x4096_rfq": (134.38208e6 + 37.032704e6) / 2}
+                     "quantize_8192x4096_rfq": (134.430976e6 + 39.872512e6) / 2}
 L2_FLUSH_BYTES = 256 << 20
 REFERENCE_RUN_SECONDS = 150.0   # host time of a whole --impl reference run
 

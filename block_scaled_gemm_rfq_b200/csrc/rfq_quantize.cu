@@ -43,7 +43,7 @@ namespace {
 
 // Launch shape and ring (compile-time; the defaults are the tuned configuration).
 #ifndef RFQ_Q_STAGES
-#define RFQ_Q_STAGES 3
+#define RFQ_Q_STAGES 2
 #endif
 #ifndef RFQ_Q_SUB
 #define RFQ_Q_SUB 1
