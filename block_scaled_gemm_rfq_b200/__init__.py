@@ -61,6 +61,7 @@ class RFQError(RuntimeError):
 
 
 def library_path() -> str:
+    """Path of the in-tree librfq.so this binding loads."""
     return _LIB_PATH
 
 
@@ -123,14 +124,17 @@ def _stream(stream):
 
 # ----------------------------------------------------------------------------- sizes
 def codes_bytes(rows: int, K: int) -> int:
+    """rfq_codes_bytes: bytes of packed E2M1 codes for [rows, K] (rows * K / 2)."""
     return int(load_library().rfq_codes_bytes(rows, K))
 
 
 def scales_bytes(rows: int, K: int) -> int:
+    """rfq_scales_bytes: bytes of E8M0 scales for [rows, K] in the MMA layout (padded to 128 rows x 4 blocks)."""
     return int(load_library().rfq_scales_bytes(rows, K))
 
 
 def linear_workspace_bytes(M: int, K: int, use_residual: bool = True) -> int:
+    """rfq_linear_workspace_bytes: workspace rfq_linear needs for an [M, K] activation."""
     return int(load_library().rfq_linear_workspace_bytes(M, K, int(bool(use_residual))))
 
 
@@ -143,6 +147,7 @@ def quantize_mxfp4(x, qx_codes, qx_scales, qr_codes=None, qr_scales=None, stream
 
 
 def quantize_weight(w, qw_codes, qw_scales, stream=None):
+    """rfq_quantize_weight on torch tensors: w [N, K] bf16 (CUDA) -> Q(W) codes and scales (no residual)."""
     N, K = w.shape
     _check(load_library().rfq_quantize_weight(_ptr(w), N, K, _ptr(qw_codes), _ptr(qw_scales), _stream(stream)),
            "rfq_quantize_weight")
@@ -158,6 +163,9 @@ def gemm(qx_codes, qx_scales, qr_codes, qr_scales, qw_codes, qw_scales, M, N, K,
 
 
 def linear(x, qw_codes, qw_scales, N, y, workspace, use_residual=True, stream=None):
+    """rfq_linear: quantize x into `workspace`, then the RFQ GEMM against the
+    pre-quantized weight (the single-kernel layer for M <= 32); y's dtype selects
+    the output type."""
     import torch
     M, K = x.shape
     y_type = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
@@ -221,6 +229,7 @@ def linear_dgrad(dy, qwt_codes, qwt_scales, K, dx, workspace, use_residual=True,
 
 
 def linear_wgrad_workspace_bytes(M: int, K: int, N: int, use_residual: bool = True) -> int:
+    """rfq_linear_wgrad_workspace_bytes: workspace of rfq_linear_wgrad for x [M, K], dy [M, N]."""
     return int(load_library().rfq_linear_wgrad_workspace_bytes(M, K, N, int(bool(use_residual))))
 
 
@@ -235,6 +244,7 @@ def linear_wgrad(x, dy, dw, workspace, use_residual=True, stream=None):
 
 
 def mxfp8_codes_bytes(rows: int, K: int) -> int:
+    """rfq_mxfp8_codes_bytes: bytes of E4M3 codes for [rows, K] (one byte per element)."""
     return int(load_library().rfq_mxfp8_codes_bytes(rows, K))
 
 
@@ -265,6 +275,8 @@ def check_device_error(stream=None):
 
 
 def debug_skip_next_fill(fill_index: int):
+    """rfq_debug_skip_next_fill: test hook; the next GEMM's first CTA skips stage
+    fill `fill_index` (its bounded wait then runs out)."""
     load_library().rfq_debug_skip_next_fill(int(fill_index))
 
 
@@ -289,6 +301,7 @@ def _empty_u8(n, device):
 
 
 def quantize_mxfp4_alloc(x, residual=True, stream=None) -> QuantizedTensor:
+    """quantize_mxfp4 into freshly allocated buffers; Q(R) too when `residual`."""
     M, K = x.shape
     cb, sb = codes_bytes(M, K), scales_bytes(M, K)
     q = QuantizedTensor(M, K, _empty_u8(cb, x.device), _empty_u8(sb, x.device),
@@ -298,6 +311,7 @@ def quantize_mxfp4_alloc(x, residual=True, stream=None) -> QuantizedTensor:
 
 
 def quantize_weight_alloc(w, stream=None) -> QuantizedTensor:
+    """quantize_weight into freshly allocated buffers."""
     N, K = w.shape
     q = QuantizedTensor(N, K, _empty_u8(codes_bytes(N, K), w.device), _empty_u8(scales_bytes(N, K), w.device))
     quantize_weight(w, q.codes, q.scales, stream)
@@ -305,6 +319,7 @@ def quantize_weight_alloc(w, stream=None) -> QuantizedTensor:
 
 
 def gemm_alloc(qa: QuantizedTensor, qw: QuantizedTensor, out_dtype=None, use_residual=True, stream=None):
+    """rfq_gemm of two QuantizedTensors into a new [qa.rows, qw.rows] tensor (bf16 unless `out_dtype`)."""
     import torch
     out_dtype = out_dtype or torch.bfloat16
     y = torch.empty((qa.rows, qw.rows), dtype=out_dtype, device=qa.codes.device)
@@ -315,6 +330,7 @@ def gemm_alloc(qa: QuantizedTensor, qw: QuantizedTensor, out_dtype=None, use_res
 
 
 def linear_fused_alloc(x, qw: QuantizedTensor, out_dtype=None, use_residual=True, stream=None):
+    """rfq_linear_fused into a new [M, qw.rows] tensor (bf16 unless `out_dtype`)."""
     import torch
     out_dtype = out_dtype or torch.bfloat16
     y = torch.empty((x.shape[0], qw.rows), dtype=out_dtype, device=x.device)
@@ -333,6 +349,7 @@ def quantize_mxfp4_t_alloc(x, residual=True, stream=None) -> QuantizedTensor:
 
 
 def linear_dgrad_alloc(dy, qwt: QuantizedTensor, out_dtype=None, use_residual=True, stream=None):
+    """rfq_linear_dgrad with a fresh workspace: dX [M, K] for dy [M, N] and Q(W^T) `qwt` (rows K)."""
     import torch
     M, N = dy.shape
     dx = torch.empty((M, qwt.rows), dtype=out_dtype or torch.bfloat16, device=dy.device)
@@ -342,6 +359,7 @@ def linear_dgrad_alloc(dy, qwt: QuantizedTensor, out_dtype=None, use_residual=Tr
 
 
 def linear_wgrad_alloc(x, dy, out_dtype=None, use_residual=True, stream=None):
+    """rfq_linear_wgrad with a fresh workspace: dW [N, K] for x [M, K] and dy [M, N]."""
     import torch
     M, K = x.shape
     N = dy.shape[1]
@@ -352,6 +370,7 @@ def linear_wgrad_alloc(x, dy, out_dtype=None, use_residual=True, stream=None):
 
 
 def quantize_mxfp8_alloc(x, stream=None) -> QuantizedTensor:
+    """quantize_mxfp8 into freshly allocated buffers."""
     M, K = x.shape
     q = QuantizedTensor(M, K, _empty_u8(mxfp8_codes_bytes(M, K), x.device), _empty_u8(scales_bytes(M, K), x.device))
     quantize_mxfp8(x, q.codes, q.scales, stream)
@@ -359,6 +378,7 @@ def quantize_mxfp8_alloc(x, stream=None) -> QuantizedTensor:
 
 
 def gemm_mxfp8_alloc(qa: QuantizedTensor, qw: QuantizedTensor, out_dtype=None, stream=None):
+    """rfq_gemm_mxfp8 of two MXFP8 QuantizedTensors into a new tensor (bf16 unless `out_dtype`)."""
     import torch
     y = torch.empty((qa.rows, qw.rows), dtype=out_dtype or torch.bfloat16, device=qa.codes.device)
     gemm_mxfp8(qa.codes, qa.scales, qw.codes, qw.scales, qa.rows, qw.rows, qa.K, y, stream)
@@ -366,6 +386,7 @@ def gemm_mxfp8_alloc(qa: QuantizedTensor, qw: QuantizedTensor, out_dtype=None, s
 
 
 def linear_alloc(x, qw: QuantizedTensor, out_dtype=None, use_residual=True, stream=None):
+    """rfq_linear with a fresh workspace and output (bf16 unless `out_dtype`)."""
     import torch
     M, K = x.shape
     out_dtype = out_dtype or torch.bfloat16
