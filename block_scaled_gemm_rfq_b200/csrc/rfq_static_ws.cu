@@ -13,7 +13,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <mutex>
 
 #include "rfq.h"
 
@@ -21,24 +20,16 @@ namespace {
 
 static __device__ __align__(256) uint8_t g_static_workspace[RFQ_STATIC_WORKSPACE_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_ws_mutex;
-void* g_ws_address[kMaxDevices] = {};   // device address of g_static_workspace, per device
-
 // Device address of the scratch array on the current device.  Host code cannot
 // use the symbol itself (on the host it names a stand-in, not device memory), so
-// the address is queried once per device, with that device current, and cached.
+// the address is looked up on every call, with the caller's device current.  The
+// lookup is a table read in the runtime; nothing is cached, so an address never
+// outlives the context it belongs to (after cudaDeviceReset the library's device
+// code is loaded again, possibly at another address).
 rfq_status_t static_workspace_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return RFQ_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return RFQ_ERR_UNSUPPORTED_DEVICE;
-  std::lock_guard<std::mutex> lock(g_ws_mutex);
-  if (g_ws_address[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr) return RFQ_ERR_CUDA;
-    g_ws_address[dev] = p;
-  }
-  *out = g_ws_address[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr) return RFQ_ERR_CUDA;
+  *out = p;
   return RFQ_OK;
 }
 
@@ -48,12 +39,17 @@ extern "C" rfq_status_t rfq_linear_static_workspace(const void* x_bf16, int64_t 
                                                     const void* qw_codes, const void* qw_scales, int64_t N,
                                                     void* y, rfq_out_t y_type, int use_residual,
                                                     cudaStream_t stream) {
+  // The argument checks come in rfq_linear's order, so both entry points return the
+  // same status for the same bad arguments; the size limit is checked last.
   if (M < 0 || N < 0 || K < 0) return RFQ_ERR_INVALID_ARG;
+  if (y_type != RFQ_OUT_F32 && y_type != RFQ_OUT_BF16) return RFQ_ERR_INVALID_ARG;
   const size_t need = rfq_linear_workspace_bytes(M, K, use_residual);
-  if (M > 0 && K > 0 && (need == 0 || need > static_cast<size_t>(RFQ_STATIC_WORKSPACE_BYTES)))
+  // Empty problems need no scratch, and shapes rfq_linear rejects (need == 0 for a
+  // bad M x K, or N not a multiple of 8) go to it unchanged for its own status.
+  if (M == 0 || N == 0 || K == 0 || need == 0 || (N % 8) != 0)
+    return rfq_linear(x_bf16, M, K, qw_codes, qw_scales, N, y, y_type, use_residual, nullptr, 0, stream);
+  if (need > static_cast<size_t>(RFQ_STATIC_WORKSPACE_BYTES))
     return RFQ_ERR_UNSUPPORTED_SHAPE;   // the quantized activation does not fit the fixed scratch array
-  if (M == 0 || N == 0) return rfq_linear(x_bf16, M, K, qw_codes, qw_scales, N, y, y_type, use_residual, nullptr, 0,
-                                          stream);
   void* ws = nullptr;
   rfq_status_t st = static_workspace_address(&ws);
   if (st != RFQ_OK) return st;

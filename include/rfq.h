@@ -267,12 +267,16 @@ rfq_status_t rfq_linear_fused(const void* x_bf16, int64_t M, int64_t K,
  * rfq_linear; the caller still provides X, the quantized weight and Y.
  *
  *   - Size limit: rfq_linear_workspace_bytes(M, K, use_residual) must not exceed
- *     RFQ_STATIC_WORKSPACE_BYTES (about M*K <= 31.5 Mi elements with the residual
- *     path, 63 Mi without); larger problems return RFQ_ERR_UNSUPPORTED_SHAPE and
- *     launch nothing.
- *   - The first call on a device looks up the array's device address on that
- *     device (once; cached afterwards).  Make that first call before any stream
- *     capture on the device.
+ *     RFQ_STATIC_WORKSPACE_BYTES.  That workspace is 1.0625 bytes per element of X
+ *     with the residual path (codes and scales of Q(X) and Q(R)) and half of that
+ *     without, plus padding, so the limit is about M*K <= 30.1 Mi elements with the
+ *     residual (e.g. 4096 x 7680) and 60.2 Mi without.  Larger problems return
+ *     RFQ_ERR_UNSUPPORTED_SHAPE and launch nothing.  Bad arguments return the
+ *     status rfq_linear returns for them.
+ *   - Every call looks up the array's device address on the current device
+ *     (nothing is cached).  On a device's first call that lookup can load this
+ *     library's device code, so make the first call on each device before any
+ *     stream capture on it.
  *   - Every call on a device shares the one array and it keeps the last call's
  *     contents.  Calls whose GPU work can overlap (different streams without
  *     ordering between them, or several host threads) race on it and corrupt
