@@ -47,12 +47,13 @@ BLOCK = 32
 
 
 def build(force: bool = False) -> str:
-    """Compile rfq_oracle.c into librfq_oracle.so (gcc, strict IEEE: no fast-math)."""
+    """Compile rfq_oracle.c into librfq_oracle.so (gcc, strict IEEE: no fast-math;
+    OpenMP spreads independent rows over the host cores and changes no result)."""
     stale = (not os.path.exists(_LIB_PATH)) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
     if force or stale:
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
         cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
-               "-ffp-contract=off", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
+               "-ffp-contract=off", "-fopenmp", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
@@ -96,6 +97,8 @@ def _load():
             lib.oracle_quantize_mxfp8_bf16.argtypes = [P, I64, I64, P, P]
             lib.oracle_dequantize_mxfp8.restype = None
             lib.oracle_dequantize_mxfp8.argtypes = [P, P, I64, I64, P]
+            lib.oracle_threads.restype = ctypes.c_int
+            lib.oracle_threads.argtypes = []
             _lib = lib
     return _lib
 
@@ -119,6 +122,11 @@ def e2m1_encode(x: float, e: int) -> int:
 def block_exponent(amax: float) -> int:
     """floor(log2 amax) - 2 clamped to [-127, 127]; -127 for 0; 128 means non-finite (0xFF)."""
     return int(_load().oracle_block_exponent(float(amax)))
+
+
+def threads() -> int:
+    """Host threads the C row loops run on (OpenMP; OMP_NUM_THREADS caps it)."""
+    return int(_load().oracle_threads())
 
 
 def bf16_value(bits: int) -> float:

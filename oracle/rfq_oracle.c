@@ -30,6 +30,9 @@
 #include <stdint.h>
 #include <stddef.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define RFQ_BLOCK 32        /* elements that share one E8M0 scale */
 #define E8M0_NAN 0xFF       /* E8M0 encoding of NaN */
@@ -164,11 +167,13 @@ void oracle_quantize_bf16(const uint16_t* x, int64_t rows, int64_t K,
                           uint8_t* codes_r, uint8_t* scales_r)
 {
     const int64_t Kb = K / RFQ_BLOCK;
-    double v[RFQ_BLOCK], r[RFQ_BLOCK];
-    uint8_t cx[RFQ_BLOCK], cr[RFQ_BLOCK];
     memset(codes_x, 0, (size_t)(rows * K / 2));
     if (codes_r) memset(codes_r, 0, (size_t)(rows * K / 2));
+    /* Rows are independent; OpenMP only spreads them over the host cores. */
+    #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < rows; ++m) {
+        double v[RFQ_BLOCK], r[RFQ_BLOCK];
+        uint8_t cx[RFQ_BLOCK], cr[RFQ_BLOCK];
         for (int64_t kb = 0; kb < Kb; ++kb) {
             const uint16_t* src = x + m * K + kb * RFQ_BLOCK;
             for (int i = 0; i < RFQ_BLOCK; ++i) v[i] = oracle_bf16_value(src[i]);
@@ -200,10 +205,11 @@ void oracle_quantize_f64(const double* x, int64_t rows, int64_t K,
                          uint8_t* codes, uint8_t* scales)
 {
     const int64_t Kb = K / RFQ_BLOCK;
-    uint8_t c[RFQ_BLOCK];
     memset(codes, 0, (size_t)(rows * K / 2));
+    #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < rows; ++m)
         for (int64_t kb = 0; kb < Kb; ++kb) {
+            uint8_t c[RFQ_BLOCK];
             uint8_t s; int e;
             quantize_block(x + m * K + kb * RFQ_BLOCK, RFQ_BLOCK, c, &s, &e);
             scales[m * Kb + kb] = s;
@@ -216,6 +222,7 @@ void oracle_quantize_f64(const double* x, int64_t rows, int64_t K,
 void oracle_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K, double* out)
 {
     const int64_t Kb = K / RFQ_BLOCK;
+    #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < rows; ++m)
         for (int64_t k = 0; k < K; ++k) {
             uint8_t s = scales[m * Kb + k / RFQ_BLOCK];
@@ -229,6 +236,7 @@ void oracle_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows
 void oracle_gemm_nt(const double* A, const double* B, int64_t M, int64_t N, int64_t K,
                     double* Y, double* absY)
 {
+    #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < M; ++i)
         for (int64_t j = 0; j < N; ++j) {
             double acc = 0.0, aacc = 0.0;
@@ -336,6 +344,7 @@ int oracle_block_exponent_e4m3(double amax)
 void oracle_quantize_mxfp8_bf16(const uint16_t* x, int64_t rows, int64_t K, uint8_t* codes, uint8_t* scales)
 {
     const int64_t Kb = K / RFQ_BLOCK;
+    #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < rows; ++m)
         for (int64_t kb = 0; kb < Kb; ++kb) {
             const uint16_t* src = x + m * K + kb * RFQ_BLOCK;
@@ -362,10 +371,21 @@ void oracle_quantize_mxfp8_bf16(const uint16_t* x, int64_t rows, int64_t K, uint
 void oracle_dequantize_mxfp8(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K, double* out)
 {
     const int64_t Kb = K / RFQ_BLOCK;
+    #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < rows; ++m)
         for (int64_t k = 0; k < K; ++k) {
             uint8_t s = scales[m * Kb + k / RFQ_BLOCK];
             double val = oracle_e4m3_value(codes[m * K + k]);
             out[m * K + k] = (s == E8M0_NAN) ? NAN : ldexp(val, (int)s - 127);
         }
+}
+
+/* Host threads the row loops above run on (1 without OpenMP). */
+int oracle_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
 }
