@@ -1,13 +1,19 @@
 """Benchmark of the RFQ MXFP4 W4A4 linear layer on B200 (one JSON line on rank 0).
 
-A step is one pass of the whole hot path on the LLM FFN up-projection workload
-(X bf16 4096 x 4096 with outlier channels and spikes, W bf16 12288 x 4096, Y bf16):
+A step is one pass of the whole hot path on the video-DiT FFN workload, the
+largest of the benchmark's workloads (X bf16 32768 x 5120, Laplace body with 8
+outlier channels; W bf16 13824 x 5120; Y bf16):
   1. rfq_quantize_weight   W -> Q(W)                       (kernel 1, no residual)
   2. rfq_quantize_mxfp4    X -> Q(X), Q(R), R = X - DQ(Q(X)) (kernel 1, fused)
   3. rfq_gemm              Y = DQ(QX) DQ(QW)^T + DQ(QR) DQ(QW)^T (kernel 2, tcgen05)
 Inputs are resident in HBM; L2 is flushed between timed steps (a 256 MiB buffer
-is written, then read back so L2 is left clean), outside the per-step CUDA events.  ``value`` is executed MMA TFLOP/s over the
-whole step (4*M*N*K per step: the residual doubles K on the tensor pipe).
+is written, then read back so L2 is left clean), outside the per-step CUDA events.
+``value`` is executed MMA TFLOP/s over the whole step (4*M*N*K per step: the
+residual doubles K on the tensor pipe).  The same line carries, as extra keys, the
+LLM FFN up-projection step (4096 x 4096 -> 12288), the quantize-only bandwidth
+workload (8192 x 4096), the GEMM with the residual off (plain MXFP4), the
+rfq_linear M sweep (M = 16 .. 16384, K = N = 4096) and the tensor-core rate of the
+GEMM's own MMA shapes measured by the library's probe.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--all-configs]
 
@@ -29,11 +35,11 @@ sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense MXFP4 : bf16 tensor throughput on B200
-# DRAM bytes (read + write) per launch from `ncu --set full` captures of the current
-# kernels (the GEMM on this FFN workload; the quantizer on 16384 x 4096, twice the
-# bench workload's units, scaled by 1/2; summaries under profiles/).  None once a
-# kernel changes.
-NCU_TRAFFIC_BYTES = {"gemm_ffn_rfq_bf16": 47.675904e6 + 61.370368e6,
+# DRAM bytes (read + write) per launch from ncu captures of the current kernels (the
+# GEMM on the FFN and DiT workloads; the quantizer on 16384 x 4096, twice the
+# bench workload's units, scaled by 1/2; summaries under profiles/).  None until
+# captured, and again once a kernel changes.
+NCU_TRAFFIC_BYTES = {"gemm_ffn_rfq_bf16": 47.675904e6 + 61.370368e6, "gemm_dit_rfq_bf16": None,
                      "quantize_8192x4096_rfq": (134.430976e6 + 39.872512e6) / 2}
 L2_FLUSH_BYTES = 256 << 20
 REFERENCE_RUN_SECONDS = 150.0   # host time of a whole --impl reference run
@@ -330,58 +336,102 @@ def quantize_bytes(M, K, residual):
     return M * K * 2 + outs * (M * K // 2 + M * K // 32)
 
 
-def run_cuda(args, rank, world, local):
-    import numpy as np
+def measure_mma_peak(rfq, local, iters=50000, launches=5):
+    """The tensor-core rate of the GEMM's own MMA shapes, operands resident in shared
+    memory (rfq_mma_rate_probe): CUDA events around each launch, the SM clock sampled
+    meanwhile, and the rate per SM clock from the kernel's clock64 span."""
     import torch
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    cycles = torch.zeros(sms, dtype=torch.int64, device="cuda")
+    out = {}
+    for variant, name, pair in ((0, "mxf4_pair", 2), (1, "mxf4_single", 1), (2, "mxf8_pair", 2)):
+        rfq.mma_rate_probe(variant, 1000, cycles)
+        torch.cuda.synchronize()
+        used = 0
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
+        with ClockSampler(local, period_s=0.005) as clk:
+            for a, b in ev:
+                a.record()
+                flops, used = rfq.mma_rate_probe(variant, iters, cycles)
+                b.record()
+            torch.cuda.synchronize()
+        rfq.check_device_error()
+        ms = [a.elapsed_time(b) for a, b in ev]
+        clusters = used // pair
+        span = int(cycles[:clusters].max().item())
+        per_clk = flops / used / span          # flops per SM per SM-clock cycle
+        c = clk.summary()
+        out[name] = {"tflops": flops / (min(ms) * 1e-3) / 1e12,
+                     "tflops_median": flops / (statistics.median(ms) * 1e-3) / 1e12,
+                     "flops_per_sm_per_clock": per_clk, "sm_mhz": c["sm_mhz"], "reasons": c["reasons"],
+                     "iterations": iters, "ms": statistics.median(ms), "sms_used": used,
+                     "tflops_all_sms_at_probe_clock": per_clk * sms * (c["sm_mhz"] or 0) * 1e6 / 1e12}
+    return out
 
-    import block_scaled_gemm_rfq_b200 as rfq
-    from block_scaled_gemm_rfq_b200 import workloads as wl
 
-    rfq.load_library()
-    peaks = load_peaks()
-    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
-    hbm_peak = peaks["hbm_gbs"]
-    flush = make_l2_flush(torch)
+def gemm_peak(peaks, probe, step_mhz, sms):
+    """Denominator of the GEMM roofline: the largest of the derived MXFP4 peak
+    (measured cuBLAS bf16 x the nominal 4x ratio), the probe's event-timed rate and the
+    probe's per-clock rate at the clock the timed GEMM ran at -- so the fraction is
+    never flattered by a low denominator."""
+    derived = peaks["bf16_tflops"] * FP4_OVER_BF16
+    cands = {"derived_bf16x4": derived}
+    if probe:
+        p = probe["mxf4_pair"]
+        cands["probe_event_timed"] = p["tflops"]
+        if step_mhz:
+            cands["probe_per_clock_at_step_clock"] = p["flops_per_sm_per_clock"] * sms * step_mhz * 1e6 / 1e12
+    basis = max(cands, key=cands.get)
+    return cands[basis], basis, cands
 
-    wk = wl.ffn_up(seed=rank)
-    M, K, N = wk.M, wk.K, wk.N
-    x, w = to_device_bf16(wk.x_bits), to_device_bf16(wk.w_bits)
-    step = RfqStep(rfq, x, w, residual=True)
-    flops = 4.0 * M * N * K
 
-    with ClockSampler(local) as clk:
-        ph = time_phases(step, args.steps, args.warmup, flush, world)
-    rfq.check_device_error()
-    step_ms_total = sum(ph["step_ms"])
-    step_ms_max = max_over_ranks(step_ms_total, world)
-    ms_per_step = step_ms_max / args.steps
-    value = world * flops * args.steps / (step_ms_max * 1e-3) / 1e12
-
-    gemm_ms = statistics.mean(ph["gemm_ms"])
-    qx_ms = statistics.mean(ph["quantize_x_ms"])
-    qw_ms = statistics.mean(ph["quantize_w_ms"])
-    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
-
-    extra = {}
-    # RFQ off (plain MXFP4): the overhead the pages call negligible
+def time_gemm_pair(rfq, x, w, flush, iters):
+    """RFQ GEMM and the same GEMM with the residual off (plain MXFP4), each alone after
+    an L2 flush: the overhead the pages call negligible."""
+    on = RfqStep(rfq, x, w, residual=True)
     off = RfqStep(rfq, x, w, residual=False)
-    off.quantize_w()
-    off.quantize_x()
-    t_off = time_kernel(off.gemm, max(10, args.steps // 2), flush)
-    t_on = time_kernel(step.gemm, max(10, args.steps // 2), flush)
-    extra["rfq_off"] = {"gemm_ms": statistics.mean(t_off), "gemm_ms_rfq": statistics.mean(t_on),
-                        "gemm_overhead": statistics.mean(t_on) / statistics.mean(t_off),
-                        "tflops_executed": 2.0 * M * N * K / (statistics.mean(t_off) * 1e-3) / 1e12}
-    del off
+    for st in (on, off):
+        st.quantize_w()
+        st.quantize_x()
+    t_off = time_kernel(off.gemm, iters, flush)
+    t_on = time_kernel(on.gemm, iters, flush)
+    M, K, N = on.M, on.K, on.N
+    rfq.check_device_error()
+    return {"gemm_ms": statistics.mean(t_off), "gemm_ms_rfq": statistics.mean(t_on),
+            "gemm_overhead": statistics.mean(t_on) / statistics.mean(t_off),
+            "tflops_executed": 2.0 * M * N * K / (statistics.mean(t_off) * 1e-3) / 1e12,
+            "tflops_executed_rfq": 4.0 * M * N * K / (statistics.mean(t_on) * 1e-3) / 1e12}
 
-    # quantize-only bandwidth workload (8192 x 4096, heavy-tailed).  Four input/output
-    # sets (X alone is 4 x 67 MB > L2) are rotated and launched back to back inside one
-    # event pair: the average launch duration.  The single launch after an L2 flush is
-    # reported beside it (it carries the fixed launch/ramp cost of an isolated kernel).
+
+def time_ffn_step(rfq, wk, flush, world, fp4_peak, steps):
+    """The LLM FFN up-projection step (4096 x 4096 -> 12288): the same three phases."""
+    x, w = to_device_bf16(wk.x_bits), to_device_bf16(wk.w_bits)
+    st = RfqStep(rfq, x, w, residual=True)
+    ph = time_phases(st, steps, 3, flush, world)
+    rfq.check_device_error()
+    M, K, N = wk.M, wk.K, wk.N
+    f = 4.0 * M * N * K
+    g = statistics.mean(ph["gemm_ms"])
+    out = {"workload": wk.name, "ms_per_step": statistics.mean(ph["step_ms"]),
+           "tflops_step": f / (statistics.mean(ph["step_ms"]) * 1e-3) / 1e12,
+           "gemm": {"ms": g, "tflops_executed": f / (g * 1e-3) / 1e12, "frac_fp4_peak": f / (g * 1e-3) / 1e12 / fp4_peak},
+           "quantize_x_ms": statistics.mean(ph["quantize_x_ms"]), "quantize_w_ms": statistics.mean(ph["quantize_w_ms"])}
+    out["rfq_off"] = time_gemm_pair(rfq, x, w, flush, 10)
+    out["rfq_off"]["frac_fp4_peak"] = out["rfq_off"]["tflops_executed"] / fp4_peak
+    return out, st
+
+
+def time_quantize_bandwidth(rfq, rank, w, flush, hbm_peak, steps):
+    """Quantize-only bandwidth workload (8192 x 4096, heavy-tailed).  Four input/output
+    sets (X alone is 4 x 67 MB > L2) are rotated and launched back to back inside one
+    event pair: the average launch duration.  The single launch after an L2 flush is
+    reported beside it (it carries the fixed launch and ramp cost of an isolated kernel)."""
+    import torch
+    from block_scaled_gemm_rfq_b200 import workloads as wl
     qb = wl.quantize_bandwidth(seed=rank)
     xq0 = to_device_bf16(qb.x_bits)
     qsets = [RfqStep(rfq, xq0 if i == 0 else xq0.clone(), w[:8], residual=True) for i in range(4)]
-    n_rot = max(40, args.steps)
+    n_rot = max(40, steps)
     for st in qsets:
         st.quantize_x()
     flush()
@@ -393,76 +443,139 @@ def run_cuda(args, rank, world, local):
     b_ev.record()
     torch.cuda.synchronize()
     q_ms = a_ev.elapsed_time(b_ev) / n_rot
-    tq = time_kernel(qsets[0].quantize_x, max(20, args.steps // 2), flush)
+    tq = time_kernel(qsets[0].quantize_x, max(20, steps // 2), flush)
+    rfq.check_device_error()
     qbytes = quantize_bytes(qb.M, qb.K, True)
     q_gbs = qbytes / (q_ms * 1e-3) / 1e9
-    extra["quantize_bandwidth"] = {"workload": qb.name, "ms": q_ms, "bytes": qbytes, "gbs": q_gbs,
-                                   "frac_hbm": q_gbs / hbm_peak, "launches": n_rot,
-                                   "timing": "4 rotated input/output sets (268 MB of X) back to back, one event pair",
-                                   "isolated_launch_ms": statistics.mean(tq),
-                                   "isolated_launch_gbs": qbytes / (statistics.mean(tq) * 1e-3) / 1e9}
-    del qsets, xq0
+    iso = statistics.mean(tq)
+    return {"workload": qb.name, "ms": q_ms, "bytes": qbytes, "gbs": q_gbs,
+            "frac_hbm": q_gbs / hbm_peak, "launches": n_rot,
+            "timing": "4 rotated input/output sets (268 MB of X) back to back, one event pair",
+            "isolated_launch_ms": iso, "isolated_launch_gbs": qbytes / (iso * 1e-3) / 1e9,
+            "isolated_launch_frac_hbm": qbytes / (iso * 1e-3) / 1e9 / hbm_peak}
 
-    if args.all_configs:
-        dk = wl.dit_ffn(seed=rank)
-        xd, wd = to_device_bf16(dk.x_bits), to_device_bf16(dk.w_bits)
+
+def time_m_sweep(rfq, rank, flush, fp4_peak, hbm_peak):
+    """rfq_linear at M in {16, ..., 16384}, K = N = 4096, RFQ and plain MXFP4: one call
+    between events after an L2 flush ("isolated"), and calls replayed back to back from a
+    CUDA graph over distinct weight/activation sets whose total exceeds L2 ("stream":
+    layer after layer, every call reads its weight from HBM).  For M <= 64 the other
+    path (quantize + GEMM, or the single-kernel layer) is timed beside it."""
+    import torch
+    from block_scaled_gemm_rfq_b200 import workloads as wl
+    sweep = {}
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    for Ms in wl.SWEEP_M:
+        sk = wl.m_sweep(Ms, seed=rank)
+        xs, ws = to_device_bf16(sk.x_bits), to_device_bf16(sk.w_bits)
+        row = {}
+        n_sets = max(2, int(2 * 126e6 // (sk.N * sk.K * 0.53 + Ms * sk.K * 2)) + 1)
         for res in (True, False):
-            s2 = RfqStep(rfq, xd, wd, residual=res)
-            s2.quantize_w()
-            s2.quantize_x()
-            t = time_kernel(s2.gemm, 10, flush)
-            f = (4.0 if res else 2.0) * dk.M * dk.N * dk.K
-            extra[f"dit_ffn_gemm_{'rfq' if res else 'off'}"] = {
-                "ms": statistics.mean(t), "tflops_executed": f / (statistics.mean(t) * 1e-3) / 1e12,
-                "frac_fp4_peak": f / (statistics.mean(t) * 1e-3) / 1e12 / fp4_peak}
-            del s2
-        del xd, wd
-        sweep = {}
-        for Ms in wl.SWEEP_M:
-            sk = wl.m_sweep(Ms, seed=rank)
-            xs, ws = to_device_bf16(sk.x_bits), to_device_bf16(sk.w_bits)
-            row = {}
-            # Layer after layer: distinct weights (and activations) per call, > 2x L2 in total.
-            n_sets = max(2, int(2 * 126e6 // (sk.N * sk.K * 0.53 + Ms * sk.K * 2)) + 1)
-            for res in (True, False):
-                qws = rfq.quantize_weight_alloc(ws)
-                y = torch.empty((Ms, sk.N), dtype=torch.bfloat16, device="cuda")
-                wsb = torch.empty(rfq.linear_workspace_bytes(Ms, sk.K, res), dtype=torch.uint8, device="cuda")
-                t = time_kernel(lambda: rfq.linear(xs, qws.codes, qws.scales, sk.N, y, wsb, res), 20, flush)
-                sets = [(xs.clone(), rfq.quantize_weight_alloc(ws),
-                         torch.empty((Ms, sk.N), dtype=torch.bfloat16, device="cuda"),
-                         torch.empty(rfq.linear_workspace_bytes(Ms, sk.K, res), dtype=torch.uint8, device="cuda"))
-                        for _ in range(n_sets)]
-                calls = [lambda a=a: rfq.linear(a[0], a[1].codes, a[1].scales, sk.N, a[2], a[3], res) for a in sets]
-                t_stream = time_stream(calls, max(2, 400 // n_sets))
-                cell = {"us": 1e3 * statistics.mean(t),
-                        "tflops_useful": 2.0 * Ms * sk.N * sk.K / (statistics.mean(t) * 1e-3) / 1e12,
-                        "us_stream": 1e3 * t_stream, "stream_sets": n_sets,
-                        "path": "fused" if Ms <= 32 else
-                                ("quantize+split-K gemm" if Ms <= 256 and (1 if Ms <= 128 else 2) * ((sk.N + 255) // 256)
-                                 < torch.cuda.get_device_properties(0).multi_processor_count // 2 else "quantize+gemm")}
-                if Ms <= rfq.FUSED_MAX_M:
-                    # the two-kernel path (quantize, then GEMM) on the same problem, for comparison
-                    s2 = RfqStep(rfq, xs, ws, residual=res)
-                    s2.quantize_w()
-                    t2 = time_kernel(lambda: (s2.quantize_x(), s2.gemm()), 20, flush)
-                    cell["two_kernel_us"] = 1e3 * statistics.mean(t2)
-                    y2 = torch.empty((Ms, sk.N), dtype=torch.bfloat16, device="cuda")
-
-                    def two(a):
+            qws = rfq.quantize_weight_alloc(ws)
+            y = torch.empty((Ms, sk.N), dtype=torch.bfloat16, device="cuda")
+            wsb = torch.empty(rfq.linear_workspace_bytes(Ms, sk.K, res), dtype=torch.uint8, device="cuda")
+            t = time_kernel(lambda: rfq.linear(xs, qws.codes, qws.scales, sk.N, y, wsb, res), 20, flush)
+            sets = [(xs.clone(), rfq.quantize_weight_alloc(ws),
+                     torch.empty((Ms, sk.N), dtype=torch.bfloat16, device="cuda"),
+                     torch.empty(rfq.linear_workspace_bytes(Ms, sk.K, res), dtype=torch.uint8, device="cuda"))
+                    for _ in range(n_sets)]
+            calls = [lambda a=a: rfq.linear(a[0], a[1].codes, a[1].scales, sk.N, a[2], a[3], res) for a in sets]
+            t_stream = time_stream(calls, max(2, 400 // n_sets))
+            f = (4.0 if res else 2.0) * Ms * sk.N * sk.K
+            w_bytes = sk.N * sk.K // 2 + rfq.scales_bytes(sk.N, sk.K)
+            io_bytes = Ms * sk.K * 2 + Ms * sk.N * 2
+            # roofline time of the layer: the slower of the MMA work at the MXFP4 peak and
+            # the weight + activation + output bytes at the HBM peak
+            t_roof = max(f / (fp4_peak * 1e12), (w_bytes + io_bytes) / (hbm_peak * 1e9))
+            cell = {"us": 1e3 * statistics.mean(t), "us_stream": 1e3 * t_stream, "stream_sets": n_sets,
+                    "tflops_useful_stream": 2.0 * Ms * sk.N * sk.K / (t_stream * 1e-3) / 1e12,
+                    "roofline_us": 1e6 * t_roof, "frac_roofline_stream": 1e6 * t_roof / (1e3 * t_stream),
+                    "path": "fused" if Ms <= 32 else
+                            ("quantize+split-K gemm" if Ms <= 256 and (1 if Ms <= 128 else 2) * ((sk.N + 255) // 256)
+                             < sms // 2 else "quantize+gemm")}
+            if Ms <= rfq.FUSED_MAX_M:
+                s2 = RfqStep(rfq, xs, ws, residual=res)
+                s2.quantize_w()
+                y2 = torch.empty((Ms, sk.N), dtype=torch.bfloat16, device="cuda")
+                if Ms <= 32:
+                    # the two-kernel path (quantize, then GEMM) on the same problem
+                    def other(a):
                         rfq.quantize_mxfp4(a[0], s2.qx_c, s2.qx_s, s2.qr_c, s2.qr_s)
                         rfq.gemm(s2.qx_c, s2.qx_s, s2.qr_c, s2.qr_s, a[1].codes, a[1].scales, Ms, sk.N, sk.K, y2)
-                    cell["two_kernel_us_stream"] = 1e3 * time_stream([lambda a=a: two(a) for a in sets],
-                                                                     max(2, 400 // n_sets))
-                    del s2
-                del sets
-                row["rfq" if res else "off"] = cell
-            sweep[str(Ms)] = row
-        extra["m_sweep_rfq_linear"] = sweep
-        extra["training_ffn"] = time_training(rfq, wk, flush, fp4_peak, hbm_peak)
-        extra["mxfp8_ffn"] = time_mxfp8(rfq, wk, flush, fp4_peak / 2.0, hbm_peak, step)
+                    name = "two_kernel_us_stream"
+                else:
+                    def other(a):   # the single-kernel layer, which rfq_linear leaves aside above 32 rows
+                        rfq.linear_fused(a[0], a[1].codes, a[1].scales, sk.N, y2, res)
+                    name = "fused_us_stream"
+                cell[name] = 1e3 * time_stream([lambda a=a: other(a) for a in sets], max(2, 400 // n_sets))
+                del s2
+            del sets
+            row["rfq" if res else "off"] = cell
+        row["rfq_overhead_stream"] = row["rfq"]["us_stream"] / row["off"]["us_stream"]
+        sweep[str(Ms)] = row
+        rfq.check_device_error()
+    return sweep
 
-    # end to end through the public API with host buffers: pinned X, W in; Y out.
+
+def run_cuda(args, rank, world, local):
+    import numpy as np
+    import torch
+
+    import block_scaled_gemm_rfq_b200 as rfq
+    from block_scaled_gemm_rfq_b200 import workloads as wl
+
+    rfq.load_library()
+    peaks = load_peaks()
+    hbm_peak = peaks["hbm_gbs"]
+    derived_fp4 = peaks["bf16_tflops"] * FP4_OVER_BF16
+    flush = make_l2_flush(torch)
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+
+    # ---- the headline step: the video-DiT FFN layer (the largest workload)
+    wk = wl.dit_ffn(seed=rank)
+    M, K, N = wk.M, wk.K, wk.N
+    x, w = to_device_bf16(wk.x_bits), to_device_bf16(wk.w_bits)
+    step = RfqStep(rfq, x, w, residual=True)
+    flops = 4.0 * M * N * K
+
+    with ClockSampler(local) as clk:
+        ph = time_phases(step, args.steps, args.warmup, flush, world)
+    rfq.check_device_error()
+    clocks = clk.summary()
+    step_ms_total = sum(ph["step_ms"])
+    step_ms_max = max_over_ranks(step_ms_total, world)
+    ms_per_step = step_ms_max / args.steps
+    value = world * flops * args.steps / (step_ms_max * 1e-3) / 1e12
+
+    gemm_ms = statistics.mean(ph["gemm_ms"])
+    qx_ms = statistics.mean(ph["quantize_x_ms"])
+    qw_ms = statistics.mean(ph["quantize_w_ms"])
+    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
+
+    extra = {}
+    # the tensor-core ceiling of the GEMM's own instruction shapes, measured here
+    probe = measure_mma_peak(rfq, local) if not args.no_probe else None
+    fp4_peak, peak_basis, peak_cands = gemm_peak(peaks, probe, clocks.get("sm_mhz"), sms)
+    if probe:
+        extra["mma_peak"] = probe
+    extra["gemm_peak_candidates_tflops"] = peak_cands
+    extra["rfq_off"] = time_gemm_pair(rfq, x, w, flush, max(5, min(10, args.steps)))
+    extra["rfq_off"]["frac_fp4_peak"] = extra["rfq_off"]["tflops_executed"] / fp4_peak
+
+    # ---- the other workloads of the benchmark, as extra keys
+    ffn, _ = time_ffn_step(rfq, wl.ffn_up(seed=rank), flush, world, fp4_peak, max(10, min(20, args.steps)))
+    extra["ffn_up"] = ffn
+    extra["quantize_bandwidth"] = time_quantize_bandwidth(rfq, rank, w, flush, hbm_peak, args.steps)
+    if not args.no_sweep:
+        extra["m_sweep_rfq_linear"] = time_m_sweep(rfq, rank, flush, fp4_peak, hbm_peak)
+    if args.all_configs:
+        fk = wl.ffn_up(seed=rank)
+        fstep = RfqStep(rfq, to_device_bf16(fk.x_bits), to_device_bf16(fk.w_bits), residual=True)
+        extra["training_ffn"] = time_training(rfq, fk, flush, fp4_peak, hbm_peak)
+        extra["mxfp8_ffn"] = time_mxfp8(rfq, fk, flush, fp4_peak / 2.0, hbm_peak, fstep)
+        del fstep
+
+    # ---- end to end through the public API with host buffers: pinned X, W in; Y out.
     # Steps stream through two device buffer sets on three streams (host->device
     # copies, compute, device->host copies), so one step's copies overlap the
     # neighbouring steps' compute and opposite-direction copies; every step still
@@ -470,7 +583,7 @@ def run_cuda(args, rank, world, local):
     xh = torch.from_numpy(wk.x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     wh = torch.from_numpy(wk.w_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     yh = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    e2e_steps = max(6, args.steps // 4)
+    e2e_steps = max(6, min(12, args.steps // 4))
     bufs = [step, RfqStep(rfq, torch.empty_like(x), torch.empty_like(w), residual=True)]
     s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()
@@ -514,8 +627,8 @@ def run_cuda(args, rank, world, local):
     b_end.record(s_in)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(a.elapsed_time(b_end), world) / e2e_steps
-    # the same, one step at a time on one stream (no overlap), for reference
-    def e2e_serial():
+
+    def e2e_serial():   # the same, one step at a time on one stream (no overlap), for reference
         x.copy_(xh, non_blocking=True)
         w.copy_(wh, non_blocking=True)
         step.run()
@@ -523,11 +636,11 @@ def run_cuda(args, rank, world, local):
     a2, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     a2.record()
-    for _ in range(e2e_steps):
+    for _ in range(3):
         e2e_serial()
     b2.record()
     torch.cuda.synchronize()
-    e2e_serial_ms = max_over_ranks(a2.elapsed_time(b2), world) / e2e_steps
+    e2e_serial_ms = max_over_ranks(a2.elapsed_time(b2), world) / 3
     if not np.array_equal(yh[0].view(torch.int16).numpy()[:4], yh[1].view(torch.int16).numpy()[:4]):
         raise RuntimeError("pipelined and serial end-to-end steps disagree")
     rfq.check_device_error()
@@ -544,20 +657,26 @@ def run_cuda(args, rank, world, local):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "mxfp4 (e2m1 x e2m1, e8m0 scales), fp32 accumulate, bf16 out",
-        "data": "synthetic (seeded numpy: N(0,1) + 0.5% outlier channels x50 + 0.01% spikes x500; W N(0,0.02))",
+        "data": "synthetic (seeded numpy: X Laplace(0,1) + 8 outlier channels x80; W N(0,0.015))",
         "config": {"workload": wk.name, "M": M, "K": K, "N": N, "rfq": True, "y": "bf16",
                    "step": "rfq_quantize_weight + rfq_quantize_mxfp4 (X, residual) + rfq_gemm",
-                   "l2": "flushed between steps (256 MiB written then read back, outside the step events)",
+                   "l2": "flushed between steps (256 MiB written then read back, outside the step events); "
+                         "the step's operands (1.5 GB) exceed L2 anyway",
                    "parallelism": f"replicas x{world}"},
         "gemm": {"ms": gemm_ms, "tflops_executed": gemm_tflops, "tflops_useful": gemm_tflops / 2,
-                 "frac_fp4_peak": gemm_tflops / fp4_peak},
-        "quantize_x": {"ms": qx_ms, "gbs": quantize_bytes(M, K, True) / (qx_ms * 1e-3) / 1e9},
-        "quantize_w": {"ms": qw_ms, "gbs": quantize_bytes(N, K, False) / (qw_ms * 1e-3) / 1e9},
-        "roofline": {"bound": "tensor", "kernel": "rfq_gemm_kernel<residual, bf16>", "achieved": gemm_tflops,
+                 "frac_fp4_peak": gemm_tflops / fp4_peak, "frac_derived_peak": gemm_tflops / derived_fp4},
+        "quantize_x": {"ms": qx_ms, "gbs": quantize_bytes(M, K, True) / (qx_ms * 1e-3) / 1e9,
+                       "frac_hbm": quantize_bytes(M, K, True) / (qx_ms * 1e-3) / 1e9 / hbm_peak},
+        "quantize_w": {"ms": qw_ms, "gbs": quantize_bytes(N, K, False) / (qw_ms * 1e-3) / 1e9,
+                       "frac_hbm": quantize_bytes(N, K, False) / (qw_ms * 1e-3) / 1e9 / hbm_peak},
+        "roofline": {"bound": "tensor", "kernel": "rfq_gemm_kernel<pair, residual, bf16>", "achieved": gemm_tflops,
                      "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
-                     "peak_basis": f"{peaks['source']} bf16_tflops {peaks['bf16_tflops']} x {FP4_OVER_BF16} "
-                                   "(nominal MXFP4:bf16 ratio), burst",
-                     "traffic": NCU_TRAFFIC_BYTES.get("gemm_ffn_rfq_bf16"), "traffic_unit": "bytes"},
+                     "peak_basis": {"derived_bf16x4": f"{peaks['source']} bf16_tflops {peaks['bf16_tflops']} x "
+                                                      f"{FP4_OVER_BF16} (nominal MXFP4:bf16 ratio), burst",
+                                    "probe_event_timed": "rfq_mma_rate_probe kind::mxf4 CTA pairs, events, this run",
+                                    "probe_per_clock_at_step_clock": "probe flops per SM clock x SMs x the step's "
+                                                                     "median SM clock"}[peak_basis],
+                     "traffic": NCU_TRAFFIC_BYTES.get("gemm_dit_rfq_bf16"), "traffic_unit": "bytes"},
         "roofline_quantize": {"bound": "hbm", "kernel": "rfq_quantize_kernel<residual>",
                               "achieved": extra["quantize_bandwidth"]["gbs"], "peak": hbm_peak, "unit": "GB/s",
                               "frac": extra["quantize_bandwidth"]["gbs"] / hbm_peak,
@@ -570,7 +689,7 @@ def run_cuda(args, rank, world, local):
                 "serial_ms_per_step": e2e_serial_ms,
                 "serial_value": world * flops / (e2e_serial_ms * 1e-3) / 1e12},
         "gpu_launches": 3 * args.steps,
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "gpu": torch.cuda.get_device_name(),
     }
     result.update(extra)
@@ -582,21 +701,24 @@ def run_cuda(args, rank, world, local):
 # ----------------------------------------------------------------------------- the oracle on the host cores
 def cpu_baseline(wk, budget_s: float):
     """The CPU oracle, as it stands, on a bounded sample of the same step, scaled to the
-    whole step: quantize n_w rows of W, m rows of X (with residual), and the float64
-    reference GEMM of those m rows against n_w columns; extrapolated by rows."""
+    whole step: quantize n_w rows of W and m rows of X (with residual) in the C oracle
+    (rows spread over the host cores), and the float64 reference GEMM of those m rows
+    against the n_w weight rows (numpy BLAS); each part is extrapolated by the rows (and,
+    for the GEMM, columns) it covers."""
     import numpy as np
 
     import oracle
     oracle.build()
     M, K, N = wk.M, wk.K, wk.N
-    m = 32
-    nw = 1024
+    m = min(M, 256)
+    nw = min(N, 1024)
+    t_start = time.perf_counter()
     t0 = time.perf_counter()
     qw = oracle.quantize_bf16(wk.w_bits[:nw], residual=False)
-    t_qw = (time.perf_counter() - t0) * (N / nw)
+    t_qw_s = time.perf_counter() - t0
     t0 = time.perf_counter()
     qa = oracle.quantize_bf16(wk.x_bits[:m], residual=True)
-    t_qx = (time.perf_counter() - t0) * (M / m)
+    t_qx_s = time.perf_counter() - t0
     A, B = oracle.rfq_operands(qa, qw, True)
     t0 = time.perf_counter()
     reps = 0
@@ -605,25 +727,35 @@ def cpu_baseline(wk, budget_s: float):
         reps += 1
         if time.perf_counter() - t0 > min(5.0, budget_s / 3):
             break
-    t_gemm = (time.perf_counter() - t0) / reps * (M / m) * (N / nw)
+    t_gemm_s = (time.perf_counter() - t0) / reps
+    sample_s = time.perf_counter() - t_start
+    t_qw, t_qx = t_qw_s * (N / nw), t_qx_s * (M / m)
+    t_gemm = t_gemm_s * (M / m) * (N / nw)
     total = t_qw + t_qx + t_gemm
     cores = len(os.sched_getaffinity(0))
+    threads = oracle.threads()
     return {"value": 4.0 * M * N * K / total / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "threads": {"quantize_c_openmp": threads, "gemm_f64_blas": cores},
+            "sample_seconds_measured": sample_s,
             "seconds_per_step_extrapolated": total,
-            "parts_s": {"quantize_w": t_qw, "quantize_x": t_qx, "gemm_f64": t_gemm},
-            "sample": f"oracle quantize of W rows [0,{nw}) and X rows [0,{m}) (C, 1 thread), float64 "
-                      f"numpy matmul of those X rows x W rows (BLAS, up to {cores} threads), "
-                      f"each scaled by rows to the full {M}x{K}x{N} step"}
+            "parts_s_extrapolated": {"quantize_w": t_qw, "quantize_x": t_qx, "gemm_f64": t_gemm},
+            "parts_s_measured": {"quantize_w": t_qw_s, "quantize_x": t_qx_s, "gemm_f64_one_rep": t_gemm_s,
+                                 "gemm_reps": reps},
+            "sample": f"oracle quantize of W rows [0,{nw}) and X rows [0,{m}) (C, OpenMP over rows, {threads} "
+                      f"threads), float64 numpy matmul of those X rows x W rows (BLAS, up to {cores} threads), "
+                      f"each part scaled by rows to the full {M}x{K}x{N} step"}
 
 
 def run_reference(args):
     """--impl reference: the oracle, timed on the host cores on this workload's bounded
-    samples, reported in the same metric/unit."""
+    samples, reported in the same metric/unit.  ``ms_per_step`` is the host time one
+    step's sample actually took; the full-step time it extrapolates to is reported
+    beside it as ``extrapolated_ms_per_full_step``."""
     from block_scaled_gemm_rfq_b200 import workloads as wl
-    wk = wl.ffn_up(seed=0)
+    wk = wl.dit_ffn(seed=0)
     # Each step's sample shrinks with the number of steps so that the whole run stays
     # near REFERENCE_RUN_SECONDS of host time (the GEMM part of a sample is timed over
-    # a third of its budget; the quantizer rows are fixed, ~0.25 s).
+    # a third of its budget; the quantizer rows are fixed, well under a second).
     budget = max(0.3, min(args.cpu_seconds, REFERENCE_RUN_SECONDS / max(1, args.steps + args.warmup)))
     samples = []
     for _ in range(args.warmup):
@@ -637,7 +769,9 @@ def run_reference(args):
         "impl": "reference",
         "metric": "RFQ W4A4 GEMM TFLOPS (% MXFP4 peak); fused RFQ quantize GB/s (% HBM)",
         "value": v, "unit": "TFLOP/s", "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * statistics.mean(s["seconds_per_step_extrapolated"] for s in samples),
+        "ms_per_step": 1e3 * statistics.mean(s["sample_seconds_measured"] for s in samples),
+        "ms_per_step_is": "host time of one step's bounded sample (measured)",
+        "extrapolated_ms_per_full_step": 1e3 * statistics.mean(s["seconds_per_step_extrapolated"] for s in samples),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
         "data": "synthetic (same seeded generator as the CUDA arm)",
         "config": {"workload": wk.name, "M": wk.M, "K": wk.K, "N": wk.N, "rfq": True, "y": "f64"},
@@ -749,8 +883,11 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
-    ap.add_argument("--all-configs", action="store_true", help="also time the DiT FFN GEMM and the M sweep")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="also time the training-side GEMMs and the MXFP8 comparator on the FFN workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-probe", action="store_true", help="skip the tensor-core rate probe")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the rfq_linear M sweep")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--kernel", choices=["quantize", "gemm", "linear", "two-kernel", "fused", "quantize-t", "gemm-yt",
                                          "quantize-mxfp8", "gemm-mxfp8"], default=None,

@@ -24,7 +24,7 @@ __all__ = [
     "quantize_mxfp4_t_alloc", "linear_wgrad_alloc", "linear_dgrad_alloc",
     "mxfp8_codes_bytes", "quantize_mxfp8", "gemm_mxfp8", "quantize_mxfp8_alloc", "gemm_mxfp8_alloc",
     "QuantizedTensor", "quantize_mxfp4_alloc", "quantize_weight_alloc", "gemm_alloc", "linear_alloc",
-    "EXPORTED_SYMBOLS", "OUT_F32", "OUT_BF16",
+    "EXPORTED_SYMBOLS", "OUT_F32", "OUT_BF16", "mma_rate_probe", "MMA_PROBE_MAX_ITERATIONS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -44,8 +44,11 @@ EXPORTED_SYMBOLS = (
     "rfq_gemm", "rfq_linear_workspace_bytes", "rfq_linear", "rfq_check_device_error", "rfq_debug_skip_next_fill",
     "rfq_linear_static_workspace", "rfq_linear_fused", "rfq_debug_fused_split", "rfq_quantize_mxfp4_t",
     "rfq_gemm_yt", "rfq_linear_dgrad", "rfq_linear_wgrad_workspace_bytes", "rfq_linear_wgrad",
-    "rfq_mxfp8_codes_bytes", "rfq_quantize_mxfp8", "rfq_gemm_mxfp8",
+    "rfq_mxfp8_codes_bytes", "rfq_quantize_mxfp8", "rfq_gemm_mxfp8", "rfq_mma_rate_probe",
 )
+
+# Largest iteration count of the tensor-core rate probe (RFQ_MMA_PROBE_MAX_ITERATIONS).
+MMA_PROBE_MAX_ITERATIONS = 100000
 
 # Size of the library's fixed scratch array (RFQ_STATIC_WORKSPACE_BYTES in include/rfq.h).
 STATIC_WORKSPACE_BYTES = 32 << 20
@@ -97,6 +100,8 @@ def load_library():
                 "rfq_mxfp8_codes_bytes": (SZ, [I64, I64]),
                 "rfq_quantize_mxfp8": (I, [P, I64, I64, P, P, P]),
                 "rfq_gemm_mxfp8": (I, [P, P, P, P, I64, I64, I64, P, I, P]),
+                "rfq_mma_rate_probe": (I, [I, I64, P, I64, ctypes.POINTER(ctypes.c_double),
+                                           ctypes.POINTER(ctypes.c_int), P]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(lib, name)
@@ -394,3 +399,16 @@ def linear_alloc(x, qw: QuantizedTensor, out_dtype=None, use_residual=True, stre
     ws = _empty_u8(linear_workspace_bytes(M, K, use_residual), x.device)
     linear(x, qw.codes, qw.scales, qw.rows, y, ws, use_residual, stream)
     return y
+
+
+def mma_rate_probe(variant, iterations, cycles, stream=None):
+    """rfq_mma_rate_probe: issue `iterations` x 8 MMAs of the GEMM's shape on every SM
+    with shared-memory-resident operands (variant 0 = kind::mxf4 CTA pairs, 1 = kind::mxf4
+    single CTAs, 2 = kind::mxf8f6f4 CTA pairs).  `cycles` is an int64 device tensor with
+    one word per cluster; returns (flops the launch executes, SMs it ran on)."""
+    flops = ctypes.c_double(0.0)
+    sms = ctypes.c_int(0)
+    _check(load_library().rfq_mma_rate_probe(int(variant), int(iterations), _ptr(cycles), cycles.numel(),
+                                             ctypes.byref(flops), ctypes.byref(sms), _stream(stream)),
+           "rfq_mma_rate_probe")
+    return flops.value, sms.value

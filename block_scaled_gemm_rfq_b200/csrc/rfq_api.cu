@@ -344,6 +344,27 @@ rfq_status_t rfq_gemm_mxfp8(const void* qx_codes, const void* qx_scales, const v
                                           y_type == RFQ_OUT_BF16, sms, g_encode_tiled, stream));
 }
 
+rfq_status_t rfq_mma_rate_probe(int variant, int64_t iterations, unsigned long long* cycles, int64_t cycles_len,
+                                double* flops, int* sms_used, cudaStream_t stream) {
+  if (variant < 0 || variant > 2 || iterations < 1 || iterations > RFQ_MMA_PROBE_MAX_ITERATIONS || !cycles ||
+      !flops || !sms_used)
+    return RFQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cycles) & 7u) != 0) return RFQ_ERR_MISALIGNED;
+  int sms = 0;
+  rfq_status_t st = current_device(&sms);
+  if (st != RFQ_OK) return st;
+  const int pair = variant == 1 ? 1 : 2;
+  const int clusters = sms / pair;
+  if (cycles_len < clusters) return RFQ_ERR_INVALID_ARG;
+  int used = 0;
+  st = from_cuda(rfq::launch_mma_rate_probe(variant, static_cast<int>(iterations), cycles, clusters, &used, stream));
+  if (st != RFQ_OK) return st;
+  const double mma_k = variant == 2 ? 32.0 : 64.0;   // K of one kind::mxf8f6f4 / kind::mxf4 MMA
+  *flops = static_cast<double>(used) * static_cast<double>(iterations) * 8.0 * 2.0 * (128.0 * pair) * 256.0 * mma_k;
+  *sms_used = used * pair;
+  return RFQ_OK;
+}
+
 rfq_status_t rfq_check_device_error(cudaStream_t stream, int* detail) {
   if (detail) *detail = 0;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return RFQ_ERR_CUDA;

@@ -569,6 +569,146 @@ cudaError_t launch_gemm_impl(const void* qx_codes, const void* qx_scales, const 
               : launch_mode<1, false>(maps, p, M, residual, y_bf16, fp8, num_sms, stream);
 }
 
+// ---------------------------------------------------------------- tensor-core rate probe
+// The MMAs of one RFQ GEMM stage issued back to back on operands that stay in
+// shared memory: no TMA, no epilogue, no pipeline waits.  What it measures is the
+// rate at which the tensor cores retire exactly the instruction shapes
+// rfq_gemm_kernel issues (kind::mxf4.block_scale, M = 128 * kPair, N = 256,
+// K = 64; or kind::mxf8f6f4, K = 32), i.e. the ceiling the GEMM's roofline
+// fraction is measured against.  Per iteration: 4 MMAs on the A tile and 4 on
+// the R tile against the same B tile, the RFQ stage's pattern.  The clock64()
+// cycles of the issuing thread (first MMA issued -> all MMAs complete) go to
+// cycles[cluster]; the caller times the launch with events as well.
+constexpr int kProbeThreads = 128;
+
+template <int kPair>
+struct ProbeLayout {
+  static constexpr uint32_t kATile = kBM * kBKBytes;             // 16 KiB
+  static constexpr uint32_t kBTile = (kBN / kPair) * kBKBytes;   // 16 or 32 KiB
+  static constexpr uint32_t kOffA = 0;
+  static constexpr uint32_t kOffR = kATile;
+  static constexpr uint32_t kOffB = 2 * kATile;
+  static constexpr uint32_t kOffSf = kOffB + kBTile;             // 4 scale atoms of 512 bytes
+  static constexpr uint32_t kOffBar = kOffSf + 2048;
+  // More shared memory than the operands need, so that no two probe CTAs share an
+  // SM (each must have the SM's tensor core to itself).
+  static constexpr uint32_t kSmem = 160u * 1024u;
+  static_assert(kOffBar + 64 + 1024 <= kSmem, "probe layout exceeds its shared memory");
+};
+
+template <int kPair, bool kFp8>
+__global__ void __launch_bounds__(kProbeThreads, 1)
+    rfq_mma_rate_kernel(int iters, unsigned long long* cycles) {
+  using L = ProbeLayout<kPair>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* done = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5;
+  const uint32_t rank = kPair == 2 ? cluster_cta_rank() : 0u;
+
+  // Operands: a fixed pseudo-random byte pattern (every E2M1 nibble is a number;
+  // E4M3 bytes are masked off the NaN codes), scale bytes 127 (2^0).
+  for (uint32_t i = threadIdx.x; i < L::kOffSf / 4; i += kProbeThreads) {
+    uint32_t h = (i + 1u) * 2654435761u;
+    h ^= h >> 15;
+    reinterpret_cast<uint32_t*>(smem)[i] = kFp8 ? (h & 0x77777777u) : h;
+  }
+  for (uint32_t i = threadIdx.x; i < 2048 / 4; i += kProbeThreads)
+    reinterpret_cast<uint32_t*>(smem + L::kOffSf)[i] = 0x7F7F7F7Fu;
+  fence_proxy_async_smem();
+  if (threadIdx.x == 0) {
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_g<kPair>(tmem_slot, kTmemCols);
+    tmem_relinquish_g<kPair>();
+  }
+  tc_fence_before();
+  if (kPair == 2) cluster_sync();   // both CTAs' operands and barriers are ready
+  else __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (threadIdx.x == 0 && rank == 0) {
+    const uint32_t sf = tmem + kSfBase;
+#pragma unroll
+    for (uint32_t a = 0; a < 4; ++a)
+      tmem_copy_32x128b_warpx4_g<kPair>(sf + 4 * a, scale_desc(smem + L::kOffSf + 512 * a));
+    const uint64_t da = operand_desc(smem + L::kOffA);
+    const uint64_t dr = operand_desc(smem + L::kOffR);
+    const uint64_t db = operand_desc(smem + L::kOffB);
+    const unsigned long long t0 = clock64();
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+      for (uint32_t q = 0; q < 4; ++q) {
+        const uint32_t id = kFp8 ? q : 2u * (q & 1u);
+        const uint32_t sfa = sf | (id << 30), sfb = (sf + 8) | (id << 30);
+        if constexpr (kFp8) mma_mxf8_g<kPair>(tmem, da + 2u * q, db + 2u * q, mma_idesc<kPair, true>(id), sfa, sfb, 1u);
+        else mma_mxf4_g<kPair>(tmem, da + 2u * q, db + 2u * q, mma_idesc<kPair, false>(id), sfa, sfb, 1u);
+      }
+#pragma unroll
+      for (uint32_t q = 0; q < 4; ++q) {
+        const uint32_t id = kFp8 ? q : 2u * (q & 1u);
+        const uint32_t sfa = (sf + 4) | (id << 30), sfb = (sf + 8) | (id << 30);
+        if constexpr (kFp8) mma_mxf8_g<kPair>(tmem, dr + 2u * q, db + 2u * q, mma_idesc<kPair, true>(id), sfa, sfb, 1u);
+        else mma_mxf4_g<kPair>(tmem, dr + 2u * q, db + 2u * q, mma_idesc<kPair, false>(id), sfa, sfb, 1u);
+      }
+    }
+    tc_commit_g<kPair>(done);
+    int never = 0;
+    mbar_wait(done, 0, &never, &g_device_error, kErrWaitDrain, 2 * kWaitLimitNs);
+    cycles[blockIdx.x / kPair] = clock64() - t0;   // grid = clusters x kPair <= cycles_len x kPair
+  } else if (threadIdx.x == 0) {
+    int never = 0;   // the peer's shared memory stays in use until the leader's MMAs complete
+    mbar_wait(done, 0, &never, &g_device_error, kErrWaitDrain, 2 * kWaitLimitNs);
+  }
+  tc_fence_before();
+  if (kPair == 2) cluster_sync();
+  else __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc_g<kPair>(tmem, kTmemCols);
+  }
+}
+
+template <int kPair, bool kFp8>
+cudaError_t launch_probe(int iters, unsigned long long* cycles, int max_clusters, int* clusters_used,
+                         cudaStream_t stream) {
+  auto kernel = rfq_mma_rate_kernel<kPair, kFp8>;
+  using L = ProbeLayout<kPair>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(max_clusters * kPair);
+  cfg.blockDim = dim3(kProbeThreads);
+  cfg.dynamicSmemBytes = L::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kPair;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // Only as many clusters as can be resident at once (one CTA per SM): a cluster that
+  // waited for a free SM pair would only add a second wave to the event time.
+  int resident = 0;
+  e = cudaOccupancyMaxActiveClusters(&resident, kernel, &cfg);
+  if (e != cudaSuccess) return e;
+  if (resident < 1) return cudaErrorInvalidConfiguration;
+  const int clusters = resident < max_clusters ? resident : max_clusters;
+  cfg.gridDim = dim3(clusters * kPair);
+  *clusters_used = clusters;
+  e = cudaLaunchKernelEx(&cfg, kernel, iters, cycles);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const void* qx_codes, const void* qx_scales, const void* qr_codes, const void* qr_scales,
@@ -584,6 +724,16 @@ cudaError_t launch_gemm_mxfp8(const void* qx_codes, const void* qx_scales, const
                               int num_sms, void* encode_tiled, cudaStream_t stream) {
   return launch_gemm_impl(qx_codes, qx_scales, nullptr, nullptr, qw_codes, qw_scales, M, N, K, y, y_bf16, false,
                           true, num_sms, encode_tiled, -1, stream);
+}
+
+cudaError_t launch_mma_rate_probe(int variant, int iters, unsigned long long* cycles, int max_clusters,
+                                  int* clusters_used, cudaStream_t stream) {
+  switch (variant) {
+    case 0: return launch_probe<2, false>(iters, cycles, max_clusters, clusters_used, stream);
+    case 1: return launch_probe<1, false>(iters, cycles, max_clusters, clusters_used, stream);
+    case 2: return launch_probe<2, true>(iters, cycles, max_clusters, clusters_used, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t read_and_clear_device_error(unsigned int* value) {

@@ -50,6 +50,14 @@ cudaError_t launch_gemm_mxfp8(const void* qx_codes, const void* qx_scales, const
                               const void* qw_scales, int64_t M, int64_t N, int64_t K, void* y, bool y_bf16,
                               int num_sms, void* encode_tiled, cudaStream_t stream);
 
+// Tensor-core rate probe: up to `max_clusters` clusters (of 2 CTAs for variants 0
+// and 2), no more than can be resident at once, issue `iters` x 8 MMAs of the
+// GEMM's shapes on shared-memory-resident operands; variant 0 = kind::mxf4 CTA
+// pair (M 256), 1 = kind::mxf4 single CTA (M 128), 2 = kind::mxf8f6f4 CTA pair.
+// cycles[cluster] = the issuing thread's clock64 span; *clusters_used = clusters launched.
+cudaError_t launch_mma_rate_probe(int variant, int iters, unsigned long long* cycles, int max_clusters,
+                                  int* clusters_used, cudaStream_t stream);
+
 // Read and clear the device error words (GEMM and quantizer) of the current device.
 cudaError_t read_and_clear_device_error(unsigned int* value);
 cudaError_t read_and_clear_quant_error(unsigned int* value);

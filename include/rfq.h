@@ -314,6 +314,35 @@ rfq_status_t rfq_gemm_mxfp8(const void* qx_codes, const void* qx_scales,
                             void* y, rfq_out_t y_type, cudaStream_t stream);
 
 /*
+ * rfq_mma_rate_probe -- measurement support (no counterpart in the paper): the rate
+ * at which this GPU's tensor cores retire the MMA instructions rfq_gemm issues,
+ * with the operands resident in shared memory (no loads, no epilogue).  It is the
+ * ceiling against which the GEMM's tensor-pipe fraction is stated.
+ *
+ *   variant     0 = kind::mxf4 block-scaled (E2M1, E8M0 per 32), CTA pair, M 256 x N 256 x K 64
+ *               1 = the same on single CTAs, M 128 x N 256 x K 64
+ *               2 = kind::mxf8f6f4 block-scaled (E4M3), CTA pair, M 256 x N 256 x K 32
+ *   iterations  1 .. RFQ_MMA_PROBE_MAX_ITERATIONS; each issues the 8 MMAs of one RFQ GEMM
+ *               stage (4 on the activation tile, 4 on the residual tile, one weight tile)
+ *   cycles      device buffer of at least cycles_len 8-byte words (8-byte aligned); word c
+ *               receives cluster c's clock64 span from its first MMA to the completion of
+ *               its last (SM clock cycles); words past the clusters launched are untouched
+ *   cycles_len  at least SM count / 2 for variants 0 and 2, the SM count for variant 1
+ *   flops       host pointer; receives the MMA flops the launch executes (2*M*N*K per MMA)
+ *   sms_used    host pointer; receives the SMs the launch ran on: one CTA per SM, and only
+ *               as many clusters as can be resident at once (on a GPU whose SM count does
+ *               not split evenly into pairs, a few SMs stay idle)
+ *
+ * Time the launch with events on `stream`; flops / time is the rate of sms_used SMs, and
+ * flops / (max cycles * sms_used) the rate per SM per clock.  The MMA results are not
+ * meaningful and nothing but `cycles` is written.  Errors: RFQ_ERR_INVALID_ARG for a bad
+ * variant, iteration count or pointer, RFQ_ERR_MISALIGNED, RFQ_ERR_UNSUPPORTED_DEVICE.
+ */
+#define RFQ_MMA_PROBE_MAX_ITERATIONS 100000
+rfq_status_t rfq_mma_rate_probe(int variant, int64_t iterations, unsigned long long* cycles, int64_t cycles_len,
+                                double* flops, int* sms_used, cudaStream_t stream);
+
+/*
  * rfq_check_device_error -- synchronize `stream`, then read and clear the current
  * device's error word that bounded waits inside the kernels set.  Returns
  * RFQ_OK, RFQ_ERR_TIMEOUT (a wait ran out; the kernel wrote no complete result),

@@ -20,8 +20,11 @@ def test_reference_arm_json_line():
     assert d["impl"] == "reference"
     assert d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
     assert d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 3
-    assert d["config"]["workload"] == "rfq_linear_ffn_up_M4096_K4096_N12288"
+    assert d["config"]["workload"] == "rfq_linear_dit_ffn_M32768_K5120_N13824"
+    # ms_per_step is the measured host time of a step's sample, not an extrapolation
+    assert 0 < d["ms_per_step"] < 60e3 and d["extrapolated_ms_per_full_step"] > d["ms_per_step"]
     cb = d["cpu_baseline"]
+    assert cb["threads"]["quantize_c_openmp"] >= 1
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 

@@ -83,6 +83,14 @@ def test_argument_errors_return_before_launch(lib):
     assert lib.rfq_debug_fused_split(9) == 1 and lib.rfq_debug_fused_split(-1) == 1
     assert lib.rfq_debug_fused_split(0) == 0
     assert lib.rfq_linear_fused(None, 0, 64, None, None, 16, None, 0, 1, None) == 0
+    # tensor-core rate probe: bad variant, iteration count, pointers, alignment
+    f, n = ctypes.c_double(0.0), ctypes.c_int(0)
+    assert lib.rfq_mma_rate_probe(3, 10, _vp(A), 1024, ctypes.byref(f), ctypes.byref(n), None) == 1
+    assert lib.rfq_mma_rate_probe(0, 0, _vp(A), 1024, ctypes.byref(f), ctypes.byref(n), None) == 1
+    assert lib.rfq_mma_rate_probe(0, 100001, _vp(A), 1024, ctypes.byref(f), ctypes.byref(n), None) == 1
+    assert lib.rfq_mma_rate_probe(0, 10, None, 1024, ctypes.byref(f), ctypes.byref(n), None) == 1
+    assert lib.rfq_mma_rate_probe(0, 10, _vp(A), 1024, None, ctypes.byref(n), None) == 1
+    assert lib.rfq_mma_rate_probe(0, 10, _vp(A + 4), 1024, ctypes.byref(f), ctypes.byref(n), None) == 3
     # empty problems are valid no-ops (no device needed)
     assert lib.rfq_quantize_mxfp4(None, 0, 64, None, None, None, None, None) == 0
     assert lib.rfq_gemm(None, None, None, None, None, None, 0, 16, 64, None, 0, None) == 0

@@ -116,57 +116,6 @@ def test_k_zero_writes_zeros(rfq):
     assert torch.count_nonzero(y).item() == 0
 
 
-def _sampled_rows_check(rfq, oracle, wk, rows, residual=True):
-    """Full-size GEMM on the GPU; the oracle recomputes the sampled rows of Y (all
-    N columns) from its own quantization of those rows of X and of all of W.
-    S is taken over the sampled rows, which is <= the full-matrix S (stricter)."""
-    import torch
-    x_sub = wk.x_bits[rows]
-    qa = oracle.quantize_bf16(x_sub, residual=residual)
-    qw = oracle.quantize_bf16(wk.w_bits, residual=False)
-    A, B = oracle.rfq_operands(qa, qw, residual)
-    Y, absY = oracle.gemm_blas(A, B)
-    S = float(absY.max())
-    for out in (torch.float32, torch.bfloat16):
-        y = run_gemm(rfq, wk.x_bits, wk.w_bits, residual, out)
-        assert_y_close(y[rows], Y, S, bf16_out=(out == torch.bfloat16), what=f"{wk.name} {out}")
-
-
-def _sample(M, n, seed):
-    rng = np.random.default_rng(seed)
-    r = set(rng.choice(M, n, replace=False).tolist()) | {0, M - 1, 127, 128}
-    return np.array(sorted(i for i in r if i < M))
-
-
-def test_ffn_up_workload_sampled(rfq, oracle):
-    wk = wl.ffn_up(0)
-    _sampled_rows_check(rfq, oracle, wk, _sample(wk.M, 60, 1))
-
-
-def test_dit_ffn_workload_sampled(rfq, oracle):
-    wk = wl.dit_ffn(0)
-    _sampled_rows_check(rfq, oracle, wk, _sample(wk.M, 24, 2), residual=True)
-
-
-def test_dit_ffn_workload_rfq_off_sampled(rfq, oracle):
-    wk = wl.dit_ffn(0)
-    _sampled_rows_check(rfq, oracle, wk, _sample(wk.M, 24, 3), residual=False)
-
-
-@pytest.mark.parametrize("M", wl.SWEEP_M)
-def test_m_sweep_linear_sampled(rfq, oracle, M):
-    import torch
-    wk = wl.m_sweep(M)
-    rows = _sample(M, min(M, 32), M)
-    for residual in (True, False):
-        qa = oracle.quantize_bf16(wk.x_bits[rows], residual=residual)
-        qw = oracle.quantize_bf16(wk.w_bits, residual=False)
-        A, B = oracle.rfq_operands(qa, qw, residual)
-        Y, absY = oracle.gemm_blas(A, B)
-        y = run_linear(rfq, wk.x_bits, wk.w_bits, residual, torch.bfloat16)
-        assert_y_close(y[rows], Y, float(absY.max()), bf16_out=True, what=f"sweep M={M} res={residual}")
-
-
 @pytest.mark.parametrize("split", [1, 2, 3, 5, 8])
 @pytest.mark.parametrize("M", [40, 200])
 def test_short_batch_gemm_every_split(rfq, oracle, split, M):
