@@ -39,7 +39,7 @@ FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense MXFP4 : bf16 tensor throughp
 # GEMM on the FFN and DiT workloads; the quantizer on 16384 x 4096, twice the
 # bench workload's units, scaled by 1/2; summaries under profiles/).  None until
 # captured, and again once a kernel changes.
-NCU_TRAFFIC_BYTES = {"gemm_ffn_rfq_bf16": 47.675904e6 + 61.370368e6, "gemm_dit_rfq_bf16": None,
+NCU_TRAFFIC_BYTES = {"gemm_ffn_rfq_bf16": 47.675904e6 + 61.370368e6, "gemm_dit_rfq_bf16": 468.86e6 + 876.77e6,
                      "quantize_8192x4096_rfq": (134.430976e6 + 39.872512e6) / 2}
 L2_FLUSH_BYTES = 256 << 20
 REFERENCE_RUN_SECONDS = 150.0   # host time of a whole --impl reference run
