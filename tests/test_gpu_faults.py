@@ -52,3 +52,35 @@ def test_skipped_fill_times_out_and_context_survives(rfq, oracle, M, N):
     rfq.check_device_error()
     Y, S, _ = oracle.rfq_linear(x_bits, w_bits, residual=True)
     assert_y_close(y_to_numpy(y2), Y, S, bf16_out=False)
+
+
+def test_short_batch_exchange_survives_an_aborted_cta(rfq, oracle):
+    """Split-K over a cluster of 4 (one k-tile each): the first CTA's only stage fill
+    is skipped, so its MMA warp's wait runs out while its three peers finish and wait
+    for it at the reduction's cluster barriers.  The aborted CTA still takes part in
+    both barriers (every thread reaches them on the error path too), so the cluster
+    completes, the error word names the stage wait, and the next call is correct."""
+    import torch
+    M, N, K = 40, 256, 1024
+    x_bits = wl.random_matrix(M, K, seed=41, scale=2.0)
+    w_bits = wl.random_matrix(N, K, seed=42, scale=0.05)
+    qa = rfq.quantize_mxfp4_alloc(dev_bf16(x_bits), residual=True)
+    qw = rfq.quantize_weight_alloc(dev_bf16(w_bits))
+    torch.cuda.synchronize()
+    rfq.check_device_error()
+    rfq.debug_skip_next_fill(0)
+    rfq.debug_fused_split(4)
+    try:
+        y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        rfq.gemm(qa.codes, qa.scales, qa.r_codes, qa.r_scales, qw.codes, qw.scales, M, N, K, y)
+        with pytest.raises(rfq.RFQError) as info:
+            rfq.check_device_error()
+        assert info.value.status == 6 and info.value.detail == 1
+        rfq.check_device_error()
+        y2 = rfq.gemm_alloc(qa, qw, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        rfq.check_device_error()
+    finally:
+        rfq.debug_fused_split(0)
+    Y, S, _ = oracle.rfq_linear(x_bits, w_bits, residual=True)
+    assert_y_close(y_to_numpy(y2), Y, S, bf16_out=False)
