@@ -12,7 +12,8 @@ is written, then read back so L2 is left clean), outside the per-step CUDA event
 residual doubles K on the tensor pipe).  The same line carries, as extra keys, the
 LLM FFN up-projection step (4096 x 4096 -> 12288), the quantize-only bandwidth
 workload (8192 x 4096), the GEMM with the residual off (plain MXFP4), the
-rfq_linear M sweep (M = 16 .. 16384, K = N = 4096), the training-side GEMMs and the
+rfq_linear M sweep (M = 16 .. 16384, K = N = 4096), the activation and output
+fidelity of RFQ against plain MXFP4 and MXFP8, the training-side GEMMs and the
 MXFP8 comparator on the FFN shape, and the tensor-core rate of the GEMM's own MMA
 shapes measured by the library's probe.
 
@@ -570,6 +571,9 @@ def run_cuda(args, rank, world, local):
     extra["quantize_bandwidth"] = time_quantize_bandwidth(rfq, rank, w, flush, hbm_peak, args.steps)
     if not args.no_sweep:
         extra["m_sweep_rfq_linear"] = time_m_sweep(rfq, rank, flush, fp4_peak, hbm_peak)
+    if not args.no_fidelity:
+        # activation and output error of RFQ, plain MXFP4 and MXFP8 on 1024 rows of each workload
+        extra["fidelity"] = run_fidelity(args)["fidelity"]
     if not args.no_training:
         # the backward-pass GEMMs and the MXFP8 comparator on the FFN workload
         fk = wl.ffn_up(seed=rank)
@@ -893,6 +897,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-probe", action="store_true", help="skip the tensor-core rate probe")
     ap.add_argument("--no-sweep", action="store_true", help="skip the rfq_linear M sweep")
+    ap.add_argument("--no-fidelity", action="store_true", help="skip the activation/output fidelity report")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--kernel", choices=["quantize", "gemm", "linear", "two-kernel", "fused", "quantize-t", "gemm-yt",
                                          "quantize-mxfp8", "gemm-mxfp8"], default=None,
