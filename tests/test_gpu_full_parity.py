@@ -82,6 +82,19 @@ def test_ffn_activation_codes_full(rfq, oracle, ffn):
     assert_quant_parity(oracle, ffn.x_bits, got, residual=True)
 
 
+@pytest.mark.parametrize("seed", [1, 2])
+def test_activation_codes_full_other_seeds(rfq, oracle, seed):
+    """The repeat-parity seeds of the FFN and DiT activations (and the FFN weight)."""
+    wk = wl.ffn_up(seed)
+    got, _ = gpu_quantize(rfq, wk.x_bits, residual=True)
+    assert_quant_parity(oracle, wk.x_bits, got, residual=True)
+    got, _ = gpu_quantize(rfq, wk.w_bits, residual=False, weight=True)
+    assert_quant_parity(oracle, wk.w_bits, got, residual=False)
+    dk = wl.dit_ffn(seed)
+    got, _ = gpu_quantize(rfq, dk.x_bits, residual=True)
+    assert_quant_parity(oracle, dk.x_bits, got, residual=True)
+
+
 def test_ffn_weight_codes_full(rfq, oracle, ffn):
     got, _ = gpu_quantize(rfq, ffn.w_bits, residual=False, weight=True)
     assert_quant_parity(oracle, ffn.w_bits, got, residual=False)
