@@ -13,7 +13,6 @@ single-CTA path (M <= 128 with enough columns to fill the GPU), the CTA-pair
 path (M > 256) and the short-batch split-K path (few tiles; K unsplit here so
 that the skipped fill is again the CTA's last) are exercised.
 """
-import numpy as np
 import pytest
 
 from block_scaled_gemm_rfq_b200 import workloads as wl

@@ -14,7 +14,6 @@ purpose.
 """
 import ctypes
 
-import numpy as np
 import pytest
 
 from block_scaled_gemm_rfq_b200 import workloads as wl
