@@ -844,6 +844,11 @@ def run_single_kernel(args):
     import block_scaled_gemm_rfq_b200 as rfq
     from block_scaled_gemm_rfq_b200 import workloads as wl
     rfq.load_library()
+    if args.kernel == "probe":
+        # the tensor-core rate of the GEMM's MMA shapes (rfq_mma_rate_probe), --steps launches each
+        dev = torch.cuda.current_device()
+        print(json.dumps({"kernel": "probe", "mma_peak": measure_mma_peak(rfq, dev, launches=max(1, args.steps))}))
+        return
     M, K, N = args.M, args.K, args.N
     x = to_device_bf16(wl.random_matrix(M, K, seed=1, scale=2.0))
     w = to_device_bf16(wl.random_matrix(N, K, seed=2, scale=0.05)) if not args.kernel.startswith("quantize") \
@@ -900,7 +905,7 @@ def main():
     ap.add_argument("--no-fidelity", action="store_true", help="skip the activation/output fidelity report")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--kernel", choices=["quantize", "gemm", "linear", "two-kernel", "fused", "quantize-t", "gemm-yt",
-                                         "quantize-mxfp8", "gemm-mxfp8"], default=None,
+                                         "quantize-mxfp8", "gemm-mxfp8", "probe"], default=None,
                     help="time one kernel on --M/--N/--K instead of the benchmark step (linear = quantize W "
                          "+ quantize X + GEMM; two-kernel = quantize X + GEMM; fused = rfq_linear_fused)")
     ap.add_argument("--split", type=int, default=0, help="with --kernel fused: K split (0 = automatic)")
