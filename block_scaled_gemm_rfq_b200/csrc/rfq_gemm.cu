@@ -68,29 +68,41 @@ constexpr uint32_t kSfaRCol = 8;       // +8+4a..:     QR
 constexpr uint32_t kSfbCol = 16;       // +16+8a..+7:  QW, the tile's 256 rows (2 row atoms)
 constexpr uint32_t kSmemLimit = 232448;
 
+// Stages of the kernels without a residual term (RFQ off, MXFP8), whose stages are a
+// third smaller: at most this many, and as many as fit.
+#ifndef RFQ_GEMM_PLAIN_STAGES
+#define RFQ_GEMM_PLAIN_STAGES 8
+#endif
+#ifndef RFQ_GEMM_PLAIN_YTILE
+#define RFQ_GEMM_PLAIN_YTILE 0
+#endif
+
 // kYTile: the epilogue stages Y in shared memory (8 warps x two 4 KiB boxes of 32
 // rows x 64 bf16, 128-byte swizzle) and stores it with TMA tensor stores; the
 // ring gives up a stage for it.  Only the RFQ kernel with CTA pairs and bf16 Y:
 // there 3 stages measured as fast as 4, while the kernels with half the MMAs per
 // stage (RFQ off, MXFP8) lost 10-13 % with 3.
 template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut, bool kFp8>
-constexpr bool kYTileFor = kPair == 2 && kResidual && kBf16Out && !kTransOut && !kFp8;
+constexpr bool kYTileFor = kPair == 2 && (kResidual || RFQ_GEMM_PLAIN_YTILE) && kBf16Out && !kTransOut && !kFp8;
 
-template <int kPair, bool kYTile = false>
+// One ring stage: the QX tile, the QR tile (residual kernels only), this CTA's part
+// of the QW tile, then the scale atoms of the same operands.
+template <int kPair, bool kResidual, bool kYTile = false>
 struct Layout {
   static constexpr uint32_t kATile = kBM * kBKBytes;                 // 16 KiB
   static constexpr uint32_t kBTile = (kBN / kPair) * kBKBytes;       // 32 KiB (single) or 16 KiB (pair)
   static constexpr uint32_t kOffA = 0;
-  static constexpr uint32_t kOffR = kOffA + kATile;
-  static constexpr uint32_t kOffB = kOffR + kATile;
+  static constexpr uint32_t kOffR = kOffA + kATile;                  // residual kernels only
+  static constexpr uint32_t kOffB = kOffA + (kResidual ? 2u : 1u) * kATile;
   static constexpr uint32_t kOffSfaX = kOffB + kBTile;               // 2 atoms (k-atom 0, 1)
-  static constexpr uint32_t kOffSfaR = kOffSfaX + 1024;
-  static constexpr uint32_t kOffSfb = kOffSfaR + 1024;               // [row atom lo, hi][k-atom 0, 1]
+  static constexpr uint32_t kOffSfaR = kOffSfaX + 1024;              // residual kernels only
+  static constexpr uint32_t kOffSfb = kOffSfaX + (kResidual ? 2048u : 1024u);   // [row atom lo, hi][k-atom 0, 1]
   static constexpr uint32_t kStage = kOffSfb + 2048;
   static constexpr uint32_t kBarrierBytes = 256;
   static constexpr uint32_t kYBox = 32 * 128;                         // 32 rows x 64 bf16
   static constexpr uint32_t kYBytes = kYTile ? 16 * kYBox : 0u;       // 8 epilogue warps x 2 boxes
-  static constexpr int kStages = static_cast<int>((kSmemLimit - 1024 - kBarrierBytes - kYBytes) / kStage);
+  static constexpr int kStagesFit = static_cast<int>((kSmemLimit - 1024 - kBarrierBytes - kYBytes) / kStage);
+  static constexpr int kStages = kResidual || kStagesFit < RFQ_GEMM_PLAIN_STAGES ? kStagesFit : RFQ_GEMM_PLAIN_STAGES;
   static constexpr uint32_t kOffY = kStages * kStage;
   static constexpr uint32_t kSmem = kStages * kStage + kYBytes + kBarrierBytes + 1024;
   static_assert(kStage % 1024 == 0, "stage buffers must keep 1 KiB alignment");
@@ -154,7 +166,7 @@ template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     rfq_gemm_kernel(const __grid_constant__ Maps maps, const GemmParams p) {
   constexpr bool kYTile = kYTileFor<kPair, kResidual, kBf16Out, kTransOut, kFp8>;
-  using L = Layout<kPair, kYTile>;
+  using L = Layout<kPair, kResidual, kYTile>;
   // A stage is 128 bytes of codes per row either way: 256 K of FP4 (2 scale atoms
   // per operand row tile) or 128 K of FP8 (1 atom).
   constexpr int kKAtoms = kFp8 ? 1 : 2;
@@ -475,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut, bool kFp8 = false>
 cudaError_t launch_typed(const Maps& maps, const GemmParams& p, int grid, cudaStream_t stream) {
   auto kernel = rfq_gemm_kernel<kPair, kResidual, kBf16Out, kTransOut, kFp8>;
-  using L = Layout<kPair, kYTileFor<kPair, kResidual, kBf16Out, kTransOut, kFp8>>;
+  using L = Layout<kPair, kResidual, kYTileFor<kPair, kResidual, kBf16Out, kTransOut, kFp8>>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
