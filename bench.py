@@ -14,8 +14,10 @@ LLM FFN up-projection step (4096 x 4096 -> 12288), the quantize-only bandwidth
 workload (8192 x 4096), the GEMM with the residual off (plain MXFP4), the
 rfq_linear M sweep (M = 16 .. 16384, K = N = 4096), the activation and output
 fidelity of RFQ against plain MXFP4 and MXFP8, the training-side GEMMs and the
-MXFP8 comparator on the FFN shape, and the tensor-core rate of the GEMM's own MMA
-shapes measured by the library's probe.
+MXFP8 comparator on the FFN shape, the tensor-core rate of the GEMM's own MMA
+shapes measured by the library's probe, and a library comparator: cuBLASLt's MXFP4
+GEMM (through torch) on the DiT step's own quantized operands, plain and with RFQ
+written as one GEMM over the operands concatenated along K.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -406,6 +408,77 @@ def time_gemm_pair(rfq, x, w, flush, iters):
             "tflops_executed_rfq": 4.0 * M * N * K / (statistics.mean(t_on) * 1e-3) / 1e12}
 
 
+def time_library_gemm(rfq, step, flush, iters):
+    """A library comparator on the step's own quantized operands: cuBLASLt's MXFP4 GEMM
+    (torch's scaled_mm, 1x32 E8M0 block scales in the 32x4x4 swizzled layout, which is
+    the layout the quantizer writes) for the plain product QX.QW^T, and for RFQ as one
+    GEMM over the operands concatenated along K ([QX | QR] . [QW | QW]^T, K' = 2K),
+    beside rfq_gemm on the same buffers; and how many bf16 outputs agree bit for bit."""
+    import torch
+    try:
+        import torch.nn.functional as F
+        BW, SW = F.ScalingType.BlockWise1x32, F.SwizzleType.SWIZZLE_32_4_4
+        fp4, e8 = torch.float4_e2m1fn_x2, torch.float8_e8m0fnu
+    except AttributeError as e:
+        return {"unavailable": f"torch has no MX scaled_mm: {e}"}
+    M, N, K = step.M, step.N, step.K
+    if K % 128:
+        return {"unavailable": "K is not a multiple of 128"}
+    Kb, rtx, rtw, kb4 = K // 2, (M + 127) // 128, (N + 127) // 128, K // 128
+
+    def lib(a, b, sa, sb, kb):
+        return F.scaled_mm(a.view(M, kb).view(fp4), b.view(N, kb).view(fp4).t(), sa.view(e8), BW, sb.view(e8), BW,
+                           swizzle_a=SW, swizzle_b=SW, output_dtype=torch.bfloat16)
+
+    cat_s = lambda s1, s2, rt: torch.cat([s1.view(rt, kb4, 512), s2.view(rt, kb4, 512)], dim=1).reshape(-1)
+    a2 = torch.cat([step.qx_c.view(M, Kb), step.qr_c.view(M, Kb)], dim=1)
+    b2 = torch.cat([step.qw_c.view(N, Kb), step.qw_c.view(N, Kb)], dim=1)
+    sa2, sb2 = cat_s(step.qx_s, step.qr_s, rtx), cat_s(step.qw_s, step.qw_s, rtw)
+    try:
+        y_lib = lib(a2, b2, sa2, sb2, 2 * Kb)
+    except Exception as e:   # no MXFP4 kernel for this device or build
+        return {"unavailable": f"scaled_mm MXFP4 failed: {repr(e)[:160]}"}
+    y_off = torch.empty_like(step.y)
+    off = lambda: step.rfq.gemm(step.qx_c, step.qx_s, None, None, step.qw_c, step.qw_s, M, N, K, y_off)
+    legs = {"rfq": step.gemm, "lib_rfq": lambda: lib(a2, b2, sa2, sb2, 2 * Kb),
+            "off": off, "lib_off": lambda: lib(step.qx_c, step.qw_c, step.qx_s, step.qw_s, Kb)}
+    for fn in legs.values():
+        fn()
+    torch.cuda.synchronize()
+    # the four legs interleaved launch by launch (an L2 flush before each), so that a
+    # change of clock or power state during the comparison affects all of them alike
+    ev = {k: [] for k in legs}
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(iters):
+            for k, fn in legs.items():
+                flush()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                fn()
+                b.record()
+                ev[k].append((a, b))
+        torch.cuda.synchronize()
+    t = {k: statistics.mean(a.elapsed_time(b) for a, b in v) for k, v in ev.items()}
+    t_rfq, t_lib_rfq, t_off, t_lib_off = t["rfq"], t["lib_rfq"], t["off"], t["lib_off"]
+    step.gemm()
+    y_lib = lib(a2, b2, sa2, sb2, 2 * Kb)
+    torch.cuda.synchronize()
+    rfq.check_device_error()
+    same = float((step.y.view(torch.int16) == y_lib.view(torch.int16)).float().mean())
+    S = float(step.y.float().abs().max())
+    diff = float((step.y.float() - y_lib.float()).abs().max()) / S
+    del a2, b2, sa2, sb2, y_lib, y_off
+    f = 2.0 * M * N * K
+    return {"library": "cuBLASLt MXFP4 through torch.nn.functional.scaled_mm", "workload": f"M{M}_K{K}_N{N}",
+            "rfq_gemm_ms": t_rfq, "library_rfq_as_2k_ms": t_lib_rfq,
+            "rfq_gemm_off_ms": t_off, "library_plain_ms": t_lib_off,
+            "rfq_speedup_vs_library": t_lib_rfq / t_rfq, "plain_speedup_vs_library": t_lib_off / t_off,
+            "rfq_tflops_executed": 2 * f / (t_rfq * 1e-3) / 1e12,
+            "library_rfq_tflops_executed": 2 * f / (t_lib_rfq * 1e-3) / 1e12,
+            "bf16_outputs_identical": same, "max_abs_diff_over_S": diff,
+            "timing": "the four legs interleaved, each launch after an L2 flush", "clocks": clk.summary()}
+
+
 def time_ffn_step(rfq, wk, flush, world, fp4_peak, steps):
     """The LLM FFN up-projection step (4096 x 4096 -> 12288): the same three phases."""
     x, w = to_device_bf16(wk.x_bits), to_device_bf16(wk.w_bits)
@@ -651,6 +724,9 @@ def run_cuda(args, rank, world, local):
     if not np.array_equal(yh[0].view(torch.int16).numpy()[:4], yh[1].view(torch.int16).numpy()[:4]):
         raise RuntimeError("pipelined and serial end-to-end steps disagree")
     rfq.check_device_error()
+    if not args.no_library:
+        # last: nothing of this run is timed after the library's kernels have run
+        extra["library_gemm"] = time_library_gemm(rfq, step, flush, max(5, min(10, args.steps)))
 
     result = {
         "metric": "RFQ W4A4 GEMM TFLOPS (% MXFP4 peak); fused RFQ quantize GB/s (% HBM)",
@@ -903,6 +979,8 @@ def main():
     ap.add_argument("--no-probe", action="store_true", help="skip the tensor-core rate probe")
     ap.add_argument("--no-sweep", action="store_true", help="skip the rfq_linear M sweep")
     ap.add_argument("--no-fidelity", action="store_true", help="skip the activation/output fidelity report")
+    ap.add_argument("--no-library", action="store_true",
+                    help="skip the library comparator (cuBLASLt MXFP4 on the step's own operands)")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--kernel", choices=["quantize", "gemm", "linear", "two-kernel", "fused", "quantize-t", "gemm-yt",
                                          "quantize-mxfp8", "gemm-mxfp8", "probe"], default=None,

@@ -26,9 +26,12 @@
 //     arithmetic as the stand-alone quantizer and write the codes into the
 //     swizzled B-operand tile and the E8M0 bytes into the stage's scale atoms in
 //     shared memory -- Q(X) and Q(R) never reach global memory;
-//   * warp 1 copies
-//     the stage's scale atoms to TMEM and issues 4 + 4 MMAs (QW.QX, QW.QR) into
-//     one fp32 accumulator of 128 lanes x Mp columns;
+//   * warp 1 copies the stage's scale atoms to TMEM and issues the MMAs.  Up to
+//     64 rows of X, Q(R)'s rows are stacked under Q(X)'s in the B tile (rows
+//     [0, Mp) and [r0, r0 + Mp), r0 = cap or 128), so 4 MMAs of N = r0 + Mp give
+//     QW.QX in accumulator columns [0, Mp) and QW.QR in [r0, r0 + Mp), added up by
+//     the epilogue; above 64 rows it issues 4 + 4 MMAs (QW.QX, QW.QR) of N = Mp
+//     into one fp32 accumulator of 128 lanes x Mp columns;
 //   * the partial accumulators of the S CTAs are summed through distributed
 //     shared memory in rank order (deterministic), each CTA reducing and
 //     storing 1/S of the tile.
@@ -69,17 +72,25 @@ constexpr unsigned int kErrWaitQuantX = 7;   // a quantizer warp waiting for its
 //   kPreQ = true (kCap = 64 or 256): Q(X), Q(R) codes and scale atoms, written
 //     before by the stand-alone quantizer, arrive by TMA like the weight tile (the
 //     short-batch GEMM: 32 < M <= 256, or any rfq_gemm call with few tiles); with
-//     up to 64 rows a stage is 35 KiB and four are in flight, with up to 256 rows
-//     it is 85 KiB and two are.
-template <int kCap, bool kPreQ>
+//     up to 64 rows a stage is 43 KiB (35 without the residual) and four are in
+//     flight, with up to 256 rows it is 85 KiB and two are.
+template <int kCap, bool kPreQ, bool kResidual>
 struct FusedLayout {
   static constexpr int kRowTiles = (kCap + 127) / 128;               // 128-row scale atoms of the activation
+  // Up to 64 rows the Q(R) rows are stacked under the Q(X) rows in one B operand
+  // of kRRow + Mp rows, Q(R) from B row kRRow (a whole number of 8-row swizzle
+  // groups): kCap when the quantizer warps build both terms' scales as one atom;
+  // 128 with pre-quantized operands, so that Q(R)'s own scale atom is copied to
+  // TMEM 4 columns after Q(X)'s (a tcgen05.cp 32x128b destination must start on
+  // a multiple of 4 columns); B rows [Mp, kRRow) are never read back.
+  static constexpr bool kStack = kResidual && kCap <= 64;
+  static constexpr int kRRow = kStack && kPreQ ? 128 : kCap;
   static constexpr int kStages = kPreQ ? (kCap <= 64 ? 4 : 2) : (kCap <= 32 ? 4 : 3);
   static constexpr uint32_t kBoxBytes = kPreQ ? 0 : kCap * 128;      // one staged box: kCap rows x 64 bf16
   static constexpr uint32_t kOffW = 0;                               // 128 x 128 B of weight codes
   static constexpr uint32_t kOffXs = kOffW + kBN * kBKBytes;         // staged X: 4 boxes (kPreQ: none)
   static constexpr uint32_t kOffX = kOffXs + 4 * kBoxBytes;          // Q(X) codes: kCap x 128 B
-  static constexpr uint32_t kOffR = kOffX + kCap * kBKBytes;         // Q(R) codes
+  static constexpr uint32_t kOffR = kOffX + kRRow * kBKBytes;        // Q(R) codes
   static constexpr uint32_t kOffSfw = kOffR + kCap * kBKBytes;       // 2 k-atoms of 512 B
   static constexpr uint32_t kOffSfx = kOffSfw + 1024;                // [row tile][k-atom] atoms of 512 B
   static constexpr uint32_t kOffSfr = kOffSfx + 1024 * kRowTiles;
@@ -89,9 +100,11 @@ struct FusedLayout {
   static constexpr uint32_t kOffRed = kPreQ ? 0 : kOffXs;
   static constexpr uint32_t kOffBar = kStages * kStage;
   static constexpr uint32_t kSmem = kOffBar + 256 + 1024;
-  // Tensor memory: the accumulator in columns [0, Mp), then one scale slot per
-  // stage: +0 QW (2 k-atoms x 4 columns), +kSfX QX and +kSfR QR (2 k-atoms x
-  // kRowTiles x 4 columns each; k-atom a, row tile t at (a * kRowTiles + t) * 4).
+  // Tensor memory: the accumulator in columns [0, Mp) (stacked terms: [0, kRRow +
+  // Mp)), then one scale slot per stage: +0 QW (2 k-atoms x 4 columns), +kSfX QX
+  // and +kSfR QR (2 k-atoms x kRowTiles x 4 columns each; k-atom a, row tile t at
+  // (a * kRowTiles + t) * 4), or, stacked, both terms' B scales of k-atom a from
+  // +kSfX + 8a.
   static constexpr uint32_t kSfBase = kPreQ ? 256 : 128;
   static constexpr uint32_t kSfSlot = kPreQ ? 64 : 32;
   static constexpr uint32_t kSfW = 0, kSfX = 8, kSfR = 8 + 8 * kRowTiles;
@@ -103,7 +116,9 @@ struct FusedLayout {
   static_assert(kStage % 1024 == 0 && kBoxBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
   static_assert(kSmem <= 232448, "exceeds the 227 KiB shared-memory limit");
   static_assert(kSfR + 8 * kRowTiles <= kSfSlot, "scale slot too small");
-  static_assert(kSfBase >= kCap && kSfBase + kStages * kSfSlot <= kTmemCols, "scale slots exceed TMEM");
+  // the accumulator: Mp <= kCap columns, or kRRow + Mp with the two terms stacked
+  static_assert(kSfBase >= (kStack ? kRRow + kCap : kCap) && kSfBase + kStages * kSfSlot <= kTmemCols,
+                "scale slots exceed TMEM");
   static_assert((4 * kStages + 2) * 8 + 8 <= 256, "barrier area too small");
 };
 
@@ -147,8 +162,10 @@ __device__ __forceinline__ uint32_t fused_idesc(uint32_t idesc_n, uint32_t sf_id
 template <int kCap, bool kResidual, bool kBf16Out, bool kPreQ>
 __global__ void __launch_bounds__(kThreads, 1)
     rfq_linear_fused_kernel(const __grid_constant__ FusedMaps maps, const FusedParams p) {
-  using L = FusedLayout<kCap, kPreQ>;
+  using L = FusedLayout<kCap, kPreQ, kResidual>;
   constexpr int kStages = L::kStages;
+  constexpr bool kStack = L::kStack;
+  constexpr int kRRow = L::kRRow;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* xfull = reinterpret_cast<uint64_t*>(smem + L::kOffBar);   // staged X landed (tx)
@@ -284,6 +301,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint8_t* st = smem + stage * L::kStage;
         const uint32_t sf = tmem + L::kSfBase + stage * L::kSfSlot;
         constexpr uint32_t kSfW = L::kSfW, kSfX = L::kSfX, kSfR = L::kSfR, kRT = L::kRowTiles;
+        if constexpr (kStack) {
+          // B scales of k-atom a from column sf + kSfX + 8a: column c holds B rows
+          // 32c .. 32c + 31.  The quantizer warps write both terms' bytes into one
+          // atom (Q(R)'s at rows kRRow = kCap ..); pre-quantized, Q(R)'s own atom goes
+          // to the 4 columns after Q(X)'s (B rows 128 .. 255).
+#pragma unroll
+          for (uint32_t a = 0; a < 2; ++a) {
+            tmem_copy_32x128b_warpx4_g<1>(sf + kSfW + 4 * a, scale_desc(st + L::kOffSfw + 512 * a));
+            tmem_copy_32x128b_warpx4_g<1>(sf + kSfX + 8 * a, scale_desc(st + L::kOffSfx + 512 * a));
+            if constexpr (kPreQ)
+              tmem_copy_32x128b_warpx4_g<1>(sf + kSfX + 8 * a + 4, scale_desc(st + L::kOffSfr + 512 * a));
+          }
+          const uint64_t dw = operand_desc(st + L::kOffW);
+          const uint64_t dx = operand_desc(st + L::kOffX);
+          const uint32_t idesc_n = static_cast<uint32_t>((kRRow + p.Mp) >> 3) << 17;
+#pragma unroll
+          for (uint32_t q = 0; q < 4; ++q) {
+            const uint32_t id = 2u * (q & 1u), a = q >> 1;
+            mma_mxf4(tmem, dw + 2u * q, dx + 2u * q, fused_idesc(idesc_n, id), (sf + kSfW + 4 * a) | (id << 30),
+                     (sf + kSfX + 8 * a) | (id << 30), (i | static_cast<int>(q)) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          continue;
+        }
 #pragma unroll
         for (uint32_t a = 0; a < 2; ++a) {
           tmem_copy_32x128b_warpx4_g<1>(sf + kSfW + 4 * a, scale_desc(st + L::kOffSfw + 512 * a));
@@ -381,7 +422,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           st[L::kOffSfx + sf_off] = static_cast<uint8_t>(sx);
           if constexpr (kResidual) {
             *reinterpret_cast<uint4*>(st + L::kOffR + code_off) = make_uint4(cr[0], cr[1], cr[2], cr[3]);
-            st[L::kOffSfr + sf_off] = static_cast<uint8_t>(sr);
+            if constexpr (kStack) {   // B row kRRow + row of the stacked operand, same atom
+              const int rr = kRRow + row;
+              st[L::kOffSfx + (j >> 2) * 512u + (rr & 31) * 16u + (rr >> 5) * 4u + (j & 3)] = static_cast<uint8_t>(sr);
+            } else {
+              st[L::kOffSfr + sf_off] = static_cast<uint8_t>(sr);
+            }
           }
         }
       }
@@ -406,6 +452,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = half; c < p.Mp / 8; c += 2) {
         uint32_t v[8];
         tmem_load_32x32b_x8(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 8 * c, v);
+        if constexpr (kStack) {   // + the Q(R) term, kRRow columns further
+          uint32_t vr[8];
+          tmem_load_32x32b_x8(tmem + (static_cast<uint32_t>(quad * 32) << 16) + kRRow + 8 * c, vr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) + __uint_as_float(vr[e]));
+        }
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -492,7 +545,7 @@ std::atomic<int> g_split_override{0};
 
 template <int kCap, bool kResidual, bool kBf16Out, bool kPreQ = false>
 cudaError_t launch_typed(const FusedMaps& maps, const FusedParams& p, int tiles, int num_sms, cudaStream_t stream) {
-  using L = FusedLayout<kCap, kPreQ>;
+  using L = FusedLayout<kCap, kPreQ, kResidual>;
   auto kernel = rfq_linear_fused_kernel<kCap, kResidual, kBf16Out, kPreQ>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
