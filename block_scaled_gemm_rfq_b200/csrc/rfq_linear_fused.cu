@@ -27,10 +27,10 @@
 //     swizzled B-operand tile and the E8M0 bytes into the stage's scale atoms in
 //     shared memory -- Q(X) and Q(R) never reach global memory;
 //   * warp 1 copies the stage's scale atoms to TMEM and issues the MMAs.  Up to
-//     64 rows of X, Q(R)'s rows are stacked under Q(X)'s in the B tile (rows
+//     128 rows of X, Q(R)'s rows are stacked under Q(X)'s in the B tile (rows
 //     [0, Mp) and [r0, r0 + Mp), r0 = cap or 128), so 4 MMAs of N = r0 + Mp give
 //     QW.QX in accumulator columns [0, Mp) and QW.QR in [r0, r0 + Mp), added up by
-//     the epilogue; above 64 rows it issues 4 + 4 MMAs (QW.QX, QW.QR) of N = Mp
+//     the epilogue; above 128 rows it issues 4 + 4 MMAs (QW.QX, QW.QR) of N = Mp
 //     into one fp32 accumulator of 128 lanes x Mp columns;
 //   * the partial accumulators of the S CTAs are summed through distributed
 //     shared memory in rank order (deterministic), each CTA reducing and
@@ -73,19 +73,19 @@ constexpr unsigned int kErrWaitQuantX = 7;   // a quantizer warp waiting for its
 //     before by the stand-alone quantizer, arrive by TMA like the weight tile (the
 //     short-batch GEMM: 32 < M <= 256, or any rfq_gemm call with few tiles); with
 //     up to 64 rows a stage is 43 KiB (35 without the residual) and four are in
-//     flight, with up to 256 rows it is 85 KiB and two are.
+//     flight, up to 128 rows 51 KiB and four, up to 256 rows 85 KiB and two.
 template <int kCap, bool kPreQ, bool kResidual>
 struct FusedLayout {
   static constexpr int kRowTiles = (kCap + 127) / 128;               // 128-row scale atoms of the activation
-  // Up to 64 rows the Q(R) rows are stacked under the Q(X) rows in one B operand
+  // Up to 128 rows the Q(R) rows are stacked under the Q(X) rows in one B operand
   // of kRRow + Mp rows, Q(R) from B row kRRow (a whole number of 8-row swizzle
   // groups): kCap when the quantizer warps build both terms' scales as one atom;
   // 128 with pre-quantized operands, so that Q(R)'s own scale atom is copied to
   // TMEM 4 columns after Q(X)'s (a tcgen05.cp 32x128b destination must start on
   // a multiple of 4 columns); B rows [Mp, kRRow) are never read back.
-  static constexpr bool kStack = kResidual && kCap <= 64;
+  static constexpr bool kStack = kResidual && kCap <= 128;
   static constexpr int kRRow = kStack && kPreQ ? 128 : kCap;
-  static constexpr int kStages = kPreQ ? (kCap <= 64 ? 4 : 2) : (kCap <= 32 ? 4 : 3);
+  static constexpr int kStages = kPreQ ? (kCap <= 128 ? 4 : 2) : (kCap <= 32 ? 4 : 3);
   static constexpr uint32_t kBoxBytes = kPreQ ? 0 : kCap * 128;      // one staged box: kCap rows x 64 bf16
   static constexpr uint32_t kOffW = 0;                               // 128 x 128 B of weight codes
   static constexpr uint32_t kOffXs = kOffW + kBN * kBKBytes;         // staged X: 4 boxes (kPreQ: none)
@@ -688,14 +688,22 @@ cudaError_t launch_gemm_short(const void* qx_codes, const void* qx_scales, const
   p.act_bytes = (static_cast<uint32_t>(Mp) * kBKBytes + row_tiles * 1024u) * (residual ? 2u : 1u);
   p.skip_fill = skip_fill;
   const int tiles = static_cast<int>((N + kBN - 1) / kBN);
-  // Up to 64 rows: 35 KiB stages, four in flight (measured 10.3 against 11.5 us per
-  // layer at M = 64, K = N = 4096, with the two-stage 85 KiB layout); up to 256: two.
+  // Up to 64 rows: four stages of 43 KiB (measured 10.3 against 11.5 us per layer
+  // at M = 64, K = N = 4096, with the two-stage 85 KiB layout, before the terms were
+  // stacked); up to 128 rows four of 51 KiB; up to 256 two.
   if (Mp <= 64) {
     if (residual)
       return y_bf16 ? launch_typed<64, true, true, true>(maps, p, tiles, num_sms, stream)
                     : launch_typed<64, true, false, true>(maps, p, tiles, num_sms, stream);
     return y_bf16 ? launch_typed<64, false, true, true>(maps, p, tiles, num_sms, stream)
                   : launch_typed<64, false, false, true>(maps, p, tiles, num_sms, stream);
+  }
+  if (Mp <= 128) {
+    if (residual)
+      return y_bf16 ? launch_typed<128, true, true, true>(maps, p, tiles, num_sms, stream)
+                    : launch_typed<128, true, false, true>(maps, p, tiles, num_sms, stream);
+    return y_bf16 ? launch_typed<128, false, true, true>(maps, p, tiles, num_sms, stream)
+                  : launch_typed<128, false, false, true>(maps, p, tiles, num_sms, stream);
   }
   if (residual)
     return y_bf16 ? launch_typed<256, true, true, true>(maps, p, tiles, num_sms, stream)
