@@ -520,15 +520,23 @@ def time_quantize_bandwidth(rfq, rank, w, flush, hbm_peak, steps):
     torch.cuda.synchronize()
     q_ms = a_ev.elapsed_time(b_ev) / n_rot
     tq = time_kernel(qsets[0].quantize_x, max(20, steps // 2), flush)
+    # the same measurement on a one-block launch of the same kernel (X 1 x 32): the fixed
+    # cost that an event pair around a single launch after the flush carries for any kernel
+    tiny = RfqStep(rfq, torch.zeros((1, 32), dtype=torch.bfloat16, device="cuda"),
+                   torch.zeros((8, 32), dtype=torch.bfloat16, device="cuda"), residual=True)
+    t_tiny = time_kernel(tiny.quantize_x, max(20, steps // 2), flush)
     rfq.check_device_error()
     qbytes = quantize_bytes(qb.M, qb.K, True)
     q_gbs = qbytes / (q_ms * 1e-3) / 1e9
-    iso = statistics.mean(tq)
+    iso, fixed = statistics.mean(tq), statistics.mean(t_tiny)
     return {"workload": qb.name, "ms": q_ms, "bytes": qbytes, "gbs": q_gbs,
             "frac_hbm": q_gbs / hbm_peak, "launches": n_rot,
             "timing": "4 rotated input/output sets (268 MB of X) back to back, one event pair",
             "isolated_launch_ms": iso, "isolated_launch_gbs": qbytes / (iso * 1e-3) / 1e9,
-            "isolated_launch_frac_hbm": qbytes / (iso * 1e-3) / 1e9 / hbm_peak}
+            "isolated_launch_frac_hbm": qbytes / (iso * 1e-3) / 1e9 / hbm_peak,
+            "one_block_launch_ms": fixed,
+            "isolated_launch_beyond_one_block_frac_hbm": qbytes / ((iso - fixed) * 1e-3) / 1e9 / hbm_peak
+            if iso > fixed else None}
 
 
 def time_m_sweep(rfq, rank, flush, fp4_peak, hbm_peak):

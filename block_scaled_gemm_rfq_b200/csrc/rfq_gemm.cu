@@ -23,14 +23,17 @@
 //               code tiles (2-D maps, 128-byte swizzle) and the stage's scale
 //               atoms (one 4-D box per operand) into a kStages-deep ring;
 //               out-of-range rows/atoms are zero-filled by the TMA unit;
-//   warp 1      MMA issuer (one thread of the leader CTA): copies the stage's
-//               scale atoms to TMEM (tcgen05.cp 32x128b.warpx4) and issues 4 + 4
-//               MMAs of K = 64; tcgen05.commit frees the stage and, at the end of
-//               a tile, signals the epilogues;
+//   warp 10     scale copies (one thread of the leader CTA): as soon as a stage
+//               has landed, copies its scale atoms to the stage's TMEM slot
+//               (tcgen05.cp 32x128b.warpx4) and commits to the stage's
+//               scales-ready barrier, running up to the ring's depth ahead of
+//               the MMAs;
+//   warp 1      MMA issuer (one thread of the leader CTA): per stage, once its
+//               scales are in TMEM, 4 + 4 MMAs of K = 64; tcgen05.commit frees the
+//               stage and, at the end of a tile, signals the epilogues;
 //   warps 2..9  epilogue: TMEM -> registers (128 columns per warp), release of
-//               the accumulator, then fp32/bf16 -> global, overlapping the next
-//               tile's mainloop: one row per thread, or (RFQ, pairs, bf16 Y)
-//               through swizzled shared-memory boxes and TMA tensor stores.
+//               the accumulator, then fp32/bf16 -> global (one row per thread),
+//               overlapping the next tile's mainloop.
 // Before its dependency wait the producer prefetches its first stages into L2.
 // Every mbarrier wait is bounded (rfq_ptx.cuh); a wait that runs out records an
 // error code, raises the CTA's abort flag and the CTA tears down cleanly.  No TMA
@@ -55,7 +58,8 @@ constexpr int kBM = 128;               // rows of X / Y per CTA (MMA M per CTA)
 constexpr int kBN = 256;               // columns of Y per tile (MMA N)
 constexpr int kBK = 256;               // K elements per stage (2 scale atoms of 128)
 constexpr int kBKBytes = kBK / 2;      // packed FP4: 128 bytes per row per stage
-constexpr int kThreads = 320;          // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kThreads = 352;          // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue, warp 10 scale copies
+constexpr int kScaleWarp = 10;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;        // 256 fp32 columns: the 128 x 256 accumulator of this CTA
 // Scale factors in TMEM: one 32-column slot per pipeline stage (from column 256),
@@ -68,26 +72,13 @@ constexpr uint32_t kSfaRCol = 8;       // +8+4a..:     QR
 constexpr uint32_t kSfbCol = 16;       // +16+8a..+7:  QW, the tile's 256 rows (2 row atoms)
 constexpr uint32_t kSmemLimit = 232448;
 
-// Stages of the kernels without a residual term (RFQ off, MXFP8), whose stages are a
-// third smaller: at most this many, and as many as fit.
-#ifndef RFQ_GEMM_PLAIN_STAGES
-#define RFQ_GEMM_PLAIN_STAGES 8
-#endif
-#ifndef RFQ_GEMM_PLAIN_YTILE
-#define RFQ_GEMM_PLAIN_YTILE 0
-#endif
-
-// kYTile: the epilogue stages Y in shared memory (8 warps x two 4 KiB boxes of 32
-// rows x 64 bf16, 128-byte swizzle) and stores it with TMA tensor stores; the
-// ring gives up a stage for it.  Only the RFQ kernel with CTA pairs and bf16 Y:
-// there 3 stages measured as fast as 4, while the kernels with half the MMAs per
-// stage (RFQ off, MXFP8) lost 10-13 % with 3.
-template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut, bool kFp8>
-constexpr bool kYTileFor = kPair == 2 && (kResidual || RFQ_GEMM_PLAIN_YTILE) && kBf16Out && !kTransOut && !kFp8;
-
 // One ring stage: the QX tile, the QR tile (residual kernels only), this CTA's part
-// of the QW tile, then the scale atoms of the same operands.
-template <int kPair, bool kResidual, bool kYTile = false>
+// of the QW tile, then the scale atoms of the same operands.  The ring holds as many
+// stages as fit: 4 for the RFQ kernel with CTA pairs (52 KiB stages), 6 for the pair
+// kernels without a residual term (35 KiB), 3 and 4 for single CTAs.  The scale warp
+// needs the depth: it copies a stage's scales as soon as the stage lands, and those
+// copies must reach the tensor pipe before the MMAs of the stage ahead of it.
+template <int kPair, bool kResidual>
 struct Layout {
   static constexpr uint32_t kATile = kBM * kBKBytes;                 // 16 KiB
   static constexpr uint32_t kBTile = (kBN / kPair) * kBKBytes;       // 32 KiB (single) or 16 KiB (pair)
@@ -99,17 +90,12 @@ struct Layout {
   static constexpr uint32_t kOffSfb = kOffSfaX + (kResidual ? 2048u : 1024u);   // [row atom lo, hi][k-atom 0, 1]
   static constexpr uint32_t kStage = kOffSfb + 2048;
   static constexpr uint32_t kBarrierBytes = 256;
-  static constexpr uint32_t kYBox = 32 * 128;                         // 32 rows x 64 bf16
-  static constexpr uint32_t kYBytes = kYTile ? 16 * kYBox : 0u;       // 8 epilogue warps x 2 boxes
-  static constexpr int kStagesFit = static_cast<int>((kSmemLimit - 1024 - kBarrierBytes - kYBytes) / kStage);
-  static constexpr int kStages = kResidual || kStagesFit < RFQ_GEMM_PLAIN_STAGES ? kStagesFit : RFQ_GEMM_PLAIN_STAGES;
-  static constexpr uint32_t kOffY = kStages * kStage;
-  static constexpr uint32_t kSmem = kStages * kStage + kYBytes + kBarrierBytes + 1024;
+  static constexpr int kStages = static_cast<int>((kSmemLimit - 1024 - kBarrierBytes) / kStage);
+  static constexpr uint32_t kSmem = kStages * kStage + kBarrierBytes + 1024;
   static_assert(kStage % 1024 == 0, "stage buffers must keep 1 KiB alignment");
   static_assert(kStages >= 3, "the ring needs at least 3 stages");
-  static_assert(kOffY % 1024 == 0, "the Y boxes need 1 KiB alignment (128-byte swizzle)");
   static_assert(kSmem <= kSmemLimit, "exceeds the 227 KiB shared-memory limit");
-  static_assert((2 * kStages + 3) * 8 + 8 <= kBarrierBytes, "barrier area too small");
+  static_assert((3 * kStages + 4) * 8 + 8 <= kBarrierBytes, "barrier area too small");
   static_assert(kSfBase + kStages * kSfSlot <= kTmemCols, "scale slots exceed TMEM");
 };
 
@@ -126,7 +112,6 @@ struct GemmParams {
 struct Maps {
   CUtensorMap x, r, w;           // codes: [rows][K/2] bytes, box 128 B x (128 | 256 | 128) rows, 128-byte swizzle
   CUtensorMap sx, sr, sw;        // scales: [row tiles][k atoms][2][256 B]; box = 2 k-atoms of 1 (A) or 2 (B) row tiles
-  CUtensorMap y;                 // Y [M][N] bf16, box 64 columns x 32 rows, 128-byte swizzle (kYTile)
 };
 
 // Shared-memory matrix descriptor (tcgen05): K-major operand, 128-byte swizzle,
@@ -165,8 +150,7 @@ __device__ __forceinline__ uint32_t mma_idesc(uint32_t sf_id) {
 template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     rfq_gemm_kernel(const __grid_constant__ Maps maps, const GemmParams p) {
-  constexpr bool kYTile = kYTileFor<kPair, kResidual, kBf16Out, kTransOut, kFp8>;
-  using L = Layout<kPair, kResidual, kYTile>;
+  using L = Layout<kPair, kResidual>;
   // A stage is 128 bytes of codes per row either way: 256 K of FP4 (2 scale atoms
   // per operand row tile) or 128 K of FP8 (1 atom).
   constexpr int kKAtoms = kFp8 ? 1 : 2;
@@ -174,12 +158,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kSfbBytes = 2u * 512u * kKAtoms;   // two row tiles (256 rows of W)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStage + L::kYBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStage);
   uint64_t* empty = full + L::kStages;
   uint64_t* acc_full = empty + L::kStages;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain_sf = drain + 1;
+  uint64_t* sready = drain_sf + 1;   // per stage: its scale atoms are in TMEM
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sready + L::kStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -197,6 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 8 * kPair);
     mbar_init(drain, 1);
+    mbar_init(drain_sf, 1);
+    for (int s = 0; s < L::kStages; ++s) mbar_init(&sready[s], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -306,22 +294,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         for (int kt = 0; kt < p.num_kt; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, &g_device_error, kErrWaitFull)) {
+          // The scale warp's commit for this stage (its copies are in TMEM), and the
+          // stage itself (already complete: the scale warp waited for it).
+          if (!mbar_wait(&sready[stage], phase, abort_flag, &g_device_error, kErrWaitFull) ||
+              !mbar_wait(&full[stage], phase, abort_flag, &g_device_error, kErrWaitFull)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint8_t* st = smem + stage * L::kStage;
           const uint32_t sf = tmem + kSfBase + stage * kSfSlot;
-#pragma unroll
-          for (uint32_t a = 0; a < kKAtoms; ++a) {
-            tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfaXCol + 4 * a, scale_desc(st + L::kOffSfaX + 512 * a));
-            if (kResidual)
-              tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfaRCol + 4 * a, scale_desc(st + L::kOffSfaR + 512 * a));
-            tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfbCol + 8 * a, scale_desc(st + L::kOffSfb + 512 * a));
-            tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfbCol + 8 * a + 4,
-                                              scale_desc(st + L::kOffSfb + 512 * kKAtoms + 512 * a));
-          }
           const uint64_t da = operand_desc(st + L::kOffA);
           const uint64_t db = operand_desc(st + L::kOffB);
           // 4 MMAs per operand over the stage's 128 bytes of K, 32 bytes each.  FP4:
@@ -363,6 +345,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(drain, 0, &never, &g_device_error, kErrWaitDrain);
       }
     }
+  } else if (warp == kScaleWarp) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------------ scale copies
+      // Same stage sequence as the MMA issuer.  A stage that has landed also has a
+      // free TMEM slot: its refill followed the MMAs' release of the stage (empty),
+      // and those were the last MMAs to read the slot.  The copies of stage s are
+      // queued while the MMAs of earlier stages still run, so the MMA thread finds
+      // them complete and issues nothing but MMAs (issuing both from one thread
+      // kept it busy for as long as the tensor pipe took for the MMAs).
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      for (int tile = unit; tile < p.num_tiles && ok; tile += num_units) {
+        for (int kt = 0; kt < p.num_kt; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, &g_device_error, kErrWaitFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* st = smem + stage * L::kStage;
+          const uint32_t sf = tmem + kSfBase + stage * kSfSlot;
+#pragma unroll
+          for (uint32_t a = 0; a < kKAtoms; ++a) {
+            tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfaXCol + 4 * a, scale_desc(st + L::kOffSfaX + 512 * a));
+            if (kResidual)
+              tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfaRCol + 4 * a, scale_desc(st + L::kOffSfaR + 512 * a));
+            tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfbCol + 8 * a, scale_desc(st + L::kOffSfb + 512 * a));
+            tmem_copy_32x128b_warpx4_g<kPair>(sf + kSfbCol + 8 * a + 4,
+                                              scale_desc(st + L::kOffSfb + 512 * kKAtoms + 512 * a));
+          }
+          tc_commit_g<kPair>(&sready[stage]);
+          if (++stage == static_cast<uint32_t>(L::kStages)) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // Teardown after an abort: wait for the copies already issued.
+        tc_commit_g<kPair>(drain_sf);
+        int never = 0;
+        mbar_wait(drain_sf, 0, &never, &g_device_error, kErrWaitDrain);
+      }
+    }
   } else {
     // -------------------------------------------------------------- epilogue
     // 8 warps: two per TMEM lane quadrant, each owning 128 of the 256 columns.
@@ -392,41 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       const int row = (mb * kPair + static_cast<int>(rank)) * kBM + quad * 32 + lane;
       const int col0 = nb * kBN + half * 128;
-      if constexpr (kYTile) {
-        // Y through shared memory and TMA: this warp's 32 rows x 128 columns as two
-        // boxes of 64 columns (128-byte rows; 16-byte chunk j of row r at position
-        // j ^ (r % 8), the 128-byte swizzle), so Y leaves in whole 128-byte row pieces
-        // instead of 16 bytes to each of 32 rows per warp store.
-        uint8_t* ybox = smem + L::kOffY + static_cast<uint32_t>(warp - 2) * 2u * L::kYBox;
-        if (lane == 0) bulk_wait_read_all();   // this warp's stores of the previous tile have read the boxes
-        __syncwarp();
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            uint32_t pw[4];
-#pragma unroll
-            for (int hh = 0; hh < 4; ++hh) {
-              const int e = 64 * cc + 8 * j + 2 * hh;
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[e >> 5][e & 31]),
-                                                        __uint_as_float(v[(e + 1) >> 5][(e + 1) & 31]));
-              pw[hh] = *reinterpret_cast<uint32_t*>(&b2);
-            }
-            *reinterpret_cast<uint4*>(ybox + cc * L::kYBox + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                make_uint4(pw[0], pw[1], pw[2], pw[3]);
-          }
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the boxes go out through TMA
-        __syncwarp();
-        if (lane == 0) {
-          const int y0 = row - lane;   // the warp's first row
-          if (y0 < p.M) {              // boxes past the end are not stored (nothing of them is in Y)
-            if (col0 < p.N) tma_store_2d(&maps.y, ybox, col0, y0);
-            if (col0 + 64 < p.N) tma_store_2d(&maps.y, ybox + L::kYBox, col0 + 64, y0);
-          }
-          bulk_commit_group();
-        }
-      } else if constexpr (kTransOut) {
+      if constexpr (kTransOut) {
         // Y^T [N][M]: for each column the warp's 32 lanes hold 32 consecutive rows,
         // so one store per column writes 32 neighbouring elements of a row of Y^T.
         if (row < p.M) {
@@ -469,9 +460,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if constexpr (kYTile) {
-      if (lane == 0) bulk_wait_all();   // Y's stores are complete before the CTA's memory goes
-    }
   }
 
   tc_fence_before();
@@ -487,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int kPair, bool kResidual, bool kBf16Out, bool kTransOut, bool kFp8 = false>
 cudaError_t launch_typed(const Maps& maps, const GemmParams& p, int grid, cudaStream_t stream) {
   auto kernel = rfq_gemm_kernel<kPair, kResidual, kBf16Out, kTransOut, kFp8>;
-  using L = Layout<kPair, kResidual, kYTileFor<kPair, kResidual, kBf16Out, kTransOut, kFp8>>;
+  using L = Layout<kPair, kResidual>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -545,19 +533,6 @@ cudaError_t launch_gemm_impl(const void* qx_codes, const void* qx_scales, const 
     return cudaErrorInvalidValue;
   if (!encode_scales_map(encode, &maps.sx, qx_scales, M, K, 1, katoms)) return cudaErrorInvalidValue;
   if (!encode_scales_map(encode, &maps.sw, qw_scales, N, K, 2, katoms)) return cudaErrorInvalidValue;
-  if (pair && y_bf16 && !y_transposed) {
-    // Y [M][N] bf16 for the TMA-store epilogue: boxes of 64 columns x 32 rows
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
-    cuuint32_t box[2] = {64u, 32u};
-    cuuint32_t elem_strides[2] = {1, 1};
-    if (encode(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, elem_strides,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  } else {
-    maps.y = maps.x;   // unused
-  }
   if (residual) {
     if (!encode_code_rows_map(encode, &maps.r, qr_codes, M, row_bytes, kBM)) return cudaErrorInvalidValue;
     if (!encode_scales_map(encode, &maps.sr, qr_scales, M, K, 1, katoms)) return cudaErrorInvalidValue;

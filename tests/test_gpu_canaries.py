@@ -2,9 +2,10 @@
 
 Each output buffer (Y, Y^T, codes, scales, workspaces) is carved out of a larger
 allocation whose first and last 4 KiB hold a known byte pattern.  After every call
-the pattern must be intact: a store past the end of an output (the clipped TMA
-boxes of the Y epilogue, the transposed quantizer's tile stores, the scale-padding
-fill, the split-K reduction stores) or before its start would change it.  The
+the pattern must be intact: a store past the end of an output (the Y epilogue's
+last row and column stores, the transposed quantizer's tile stores, the
+scale-padding fill, the split-K reduction stores) or before its start would change
+it.  The
 shapes are ragged in M and N (and K where the path allows) so that the stores near
 the ends of the buffers are exercised.  Every call's result is also checked against
 the oracle (Y within 1e-5 * S, codes and scales bit for bit), so a guard that stays
@@ -88,7 +89,7 @@ def test_weight_quantizer_guards(rfq, oracle):
 
 
 # (M, N, K): (100, 19200, 256) single-CTA tiled kernel with many tiles; (300, 520, 1024)
-# CTA pairs with ragged M and N (bf16: the TMA-store epilogue's clipped boxes);
+# CTA pairs with ragged M and N (the epilogue's guarded row and column stores);
 # (40, 384, 2304), (96, 520, 2304) and (200, 264, 2304) the short-batch split-K
 # kernel in its three layouts (ragged reduction slices); (1000, 72, 256) a single
 # ragged column tile.

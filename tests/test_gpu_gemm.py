@@ -67,8 +67,7 @@ def test_tiny_bf16_output(rfq, oracle):
                                    (1000, 72, 256)])
 @pytest.mark.parametrize("residual", [True, False])
 def test_edge_shapes(rfq, oracle, M, N, K, residual):
-    """fp32 and bf16 Y (bf16 with CTA pairs and the residual goes through the
-    TMA-store epilogue, whose boxes are clipped at ragged M and N)."""
+    """fp32 and bf16 Y, ragged M, N and K on every GEMM path."""
     import torch
     x = wl.random_matrix(M, K, seed=M + 3 * N + 7 * K, scale=2.0)
     w = wl.random_matrix(N, K, seed=M * N + K, scale=0.05)
