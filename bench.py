@@ -43,7 +43,7 @@ FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense MXFP4 : bf16 tensor throughp
 # GEMM on the FFN and DiT workloads; the quantizer on 16384 x 4096, twice the
 # bench workload's units, scaled by 1/2; summaries under profiles/).  None until
 # captured, and again once a kernel changes.
-NCU_TRAFFIC_BYTES = {"gemm_ffn_rfq_bf16": 47.675904e6 + 61.370368e6, "gemm_dit_rfq_bf16": 468.86e6 + 876.77e6,
+NCU_TRAFFIC_BYTES = {"gemm_ffn_rfq_bf16": 46.665472e6 + 53.230336e6, "gemm_dit_rfq_bf16": 470.674176e6 + 872.390656e6,
                      "quantize_8192x4096_rfq": (134.430976e6 + 39.872512e6) / 2}
 L2_FLUSH_BYTES = 256 << 20
 REFERENCE_RUN_SECONDS = 150.0   # host time of a whole --impl reference run
@@ -82,7 +82,8 @@ class ClockSampler:
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
     def __init__(self, device_index: int, period_s: float = 0.01):
-        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.samples, self.reasons, self.max_mhz, self.power_w = [], set(), None, []
+        self.handle_by = None
         self._stop = threading.Event()
         self._period = period_s
         try:
@@ -95,20 +96,23 @@ class ClockSampler:
             self._nvml = None
         self._t = threading.Thread(target=self._run, daemon=True)
 
-    @staticmethod
-    def _handle(pynvml, device_index):
+    def _handle(self, pynvml, device_index):
         # NVML enumerates every GPU of the machine; find the one torch uses by UUID
         try:
             import torch
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
-            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.handle_by = "uuid"
+            return h
         except Exception:
+            self.handle_by = "index"
             return pynvml.nvmlDeviceGetHandleByIndex(device_index)
 
     def _run(self):
         while not self._stop.is_set():
             try:
                 self.samples.append(self._nvml.nvmlDeviceGetClockInfo(self._h, self._nvml.NVML_CLOCK_SM))
+                self.power_w.append(self._nvml.nvmlDeviceGetPowerUsage(self._h) / 1000.0)
                 r = self._nvml.nvmlDeviceGetCurrentClocksEventReasons(self._h)
                 for bit, name in self.REASONS.items():
                     if r & bit:
@@ -131,7 +135,9 @@ class ClockSampler:
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples),
+                "power_w_median": statistics.median(self.power_w) if self.power_w else None,
+                "power_w_max": max(self.power_w) if self.power_w else None, "nvml_device_by": self.handle_by}
 
 
 # ----------------------------------------------------------------------------- distributed plumbing
