@@ -26,12 +26,14 @@
 //     arithmetic as the stand-alone quantizer and write the codes into the
 //     swizzled B-operand tile and the E8M0 bytes into the stage's scale atoms in
 //     shared memory -- Q(X) and Q(R) never reach global memory;
-//   * warp 1 copies the stage's scale atoms to TMEM and issues the MMAs.  Up to
-//     128 rows of X, Q(R)'s rows are stacked under Q(X)'s in the B tile (rows
-//     [0, Mp) and [r0, r0 + Mp), r0 = cap or 128), so 4 MMAs of N = r0 + Mp give
-//     QW.QX in accumulator columns [0, Mp) and QW.QR in [r0, r0 + Mp), added up by
-//     the epilogue; above 128 rows it issues 4 + 4 MMAs (QW.QX, QW.QR) of N = Mp
-//     into one fp32 accumulator of 128 lanes x Mp columns;
+//   * warp 1 copies the stage's scale atoms to TMEM and issues the MMAs: Q(R)'s
+//     rows are stacked under Q(X)'s in the B tile (rows [0, Mp) and [r0, r0 + Mp),
+//     r0 = cap or 128), so 4 MMAs of N = r0 + Mp give QW.QX in accumulator columns
+//     [0, Mp) and QW.QR in [r0, r0 + Mp), added up by the epilogue (without the
+//     residual, 4 MMAs of N = Mp);
+//   * above 128 rows (pre-quantized operands), X is taken in blocks of 128 rows,
+//     one grid row per block and weight tile, so each CTA's partial tile covers
+//     128 rows;
 //   * the partial accumulators of the S CTAs are summed through distributed
 //     shared memory in rank order (deterministic), each CTA reducing and
 //     storing 1/S of the tile.
@@ -69,11 +71,11 @@ constexpr unsigned int kErrWaitQuantX = 7;   // a quantizer warp waiting for its
 // Shared memory and tensor memory of one CTA for at most kCap rows of X.
 //   kPreQ = false (kCap = 32 or 64): X arrives as bf16 and the quantizer warps
 //     write Q(X), Q(R) into the stage;
-//   kPreQ = true (kCap = 64 or 256): Q(X), Q(R) codes and scale atoms, written
+//   kPreQ = true (kCap = 64 or 128): Q(X), Q(R) codes and scale atoms, written
 //     before by the stand-alone quantizer, arrive by TMA like the weight tile (the
-//     short-batch GEMM: 32 < M <= 256, or any rfq_gemm call with few tiles); with
-//     up to 64 rows a stage is 43 KiB (35 without the residual) and four are in
-//     flight, up to 128 rows 51 KiB and four, up to 256 rows 85 KiB and two.
+//     short-batch GEMM: 32 < M <= 256, or any rfq_gemm call with few tiles; above
+//     128 rows each CTA takes one 128-row block of X); with up to 64 rows a stage
+//     is 43 KiB (35 without the residual), with 128 rows 51 KiB; four in flight.
 template <int kCap, bool kPreQ, bool kResidual>
 struct FusedLayout {
   static constexpr int kRowTiles = (kCap + 127) / 128;               // 128-row scale atoms of the activation
@@ -133,6 +135,7 @@ struct FusedParams {
   int group;           // k-tiles quantized per round
   uint32_t idesc_n;    // (Mp / 8) << 17
   uint32_t act_bytes;  // kPreQ: bytes of Q(X) [+ Q(R)] codes and scale atoms per stage
+  int row_blocks;      // blocks of kCap rows of X, each a grid row of its own (kPreQ, 128 < M <= 256: 2)
   int skip_fill;       // kPreQ fault injection: CTA (0, 0) skips this stage fill (-1 = off)
 };
 
@@ -182,7 +185,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int split = static_cast<int>(gridDim.x);              // cluster size along K
   const uint32_t rank = cluster_cta_rank();                   // = blockIdx.x
-  const int tile = static_cast<int>(blockIdx.y);
+  // Grid rows: weight tiles x row blocks of X (row block fastest, so the clusters of
+  // neighbouring rows share the weight tile in L2).  This CTA's rows of X: [m0, m0 + mp),
+  // mp a multiple of 16; rows at and past M (m_end) are zero-filled and not stored.
+  const int rb = static_cast<int>(blockIdx.y) % p.row_blocks;
+  const int tile = static_cast<int>(blockIdx.y) / p.row_blocks;
+  const int m0 = rb * kCap;
+  const int mp = min(p.Mp - m0, kCap);
+  const int m_end = p.M - m0;
   const int n0 = tile * kBN;
   const int kt0 = static_cast<int>(rank) * p.num_kt / split;
   const int nk = (static_cast<int>(rank) + 1) * p.num_kt / split - kt0;   // >= 1: split <= num_kt
@@ -202,11 +212,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (i == p.skip_fill && blockIdx.x == 0 && blockIdx.y == 0) return;   // fault injection (tests)
       // weight tile and the activation's codes and scale atoms, all on one barrier
       mbar_arrive_expect_tx(&wfull[stage], kBN * kBKBytes + 1024u + p.act_bytes);
-      tma_load_2d(st + L::kOffX, &maps.qx, &wfull[stage], kt * kBKBytes, 0);
-      tma_load_4d(st + L::kOffSfx, &maps.sx, &wfull[stage], 0, 0, 2 * kt, 0);
+      tma_load_2d(st + L::kOffX, &maps.qx, &wfull[stage], kt * kBKBytes, m0);
+      tma_load_4d(st + L::kOffSfx, &maps.sx, &wfull[stage], 0, 0, 2 * kt, rb);
       if (kResidual) {
-        tma_load_2d(st + L::kOffR, &maps.qr, &wfull[stage], kt * kBKBytes, 0);
-        tma_load_4d(st + L::kOffSfr, &maps.sr, &wfull[stage], 0, 0, 2 * kt, 0);
+        tma_load_2d(st + L::kOffR, &maps.qr, &wfull[stage], kt * kBKBytes, m0);
+        tma_load_4d(st + L::kOffSfr, &maps.sr, &wfull[stage], 0, 0, 2 * kt, rb);
       }
     } else {
       mbar_arrive_expect_tx(&xfull[stage], x_bytes);
@@ -315,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint64_t dw = operand_desc(st + L::kOffW);
           const uint64_t dx = operand_desc(st + L::kOffX);
-          const uint32_t idesc_n = static_cast<uint32_t>((kRRow + p.Mp) >> 3) << 17;
+          const uint32_t idesc_n = static_cast<uint32_t>((kRRow + mp) >> 3) << 17;
 #pragma unroll
           for (uint32_t q = 0; q < 4; ++q) {
             const uint32_t id = 2u * (q & 1u), a = q >> 1;
@@ -449,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int half = (warp - 2) >> 2;
       const int n_local = quad * 32 + lane;
       const int n = n0 + n_local;
-      for (int c = half; c < p.Mp / 8; c += 2) {
+      for (int c = half; c < mp / 8; c += 2) {
         uint32_t v[8];
         tmem_load_32x32b_x8(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 8 * c, v);
         if constexpr (kStack) {   // + the Q(R) term, kRRow columns further
@@ -465,11 +475,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int m = 8 * c + e;
           if (split > 1) {
             red[m * kBN + n_local] = __uint_as_float(v[e]);
-          } else if (m < p.M && n < p.N) {
+          } else if (m < m_end && n < p.N) {
             if (kBf16Out)
-              static_cast<__nv_bfloat16*>(p.y)[static_cast<int64_t>(m) * p.N + n] = __float2bfloat16_rn(__uint_as_float(v[e]));
+              static_cast<__nv_bfloat16*>(p.y)[static_cast<int64_t>(m0 + m) * p.N + n] = __float2bfloat16_rn(__uint_as_float(v[e]));
             else
-              static_cast<float*>(p.y)[static_cast<int64_t>(m) * p.N + n] = __uint_as_float(v[e]);
+              static_cast<float*>(p.y)[static_cast<int64_t>(m0 + m) * p.N + n] = __uint_as_float(v[e]);
           }
         }
       }
@@ -489,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     cluster_sync();
     constexpr int kPer = kCap / 16;            // >= ceil(F / split / kQThreads) for split >= 2
     float4 acc[kPer];
-    const int F = p.Mp * (kBN / 4);            // float4 groups in the tile
+    const int F = mp * (kBN / 4);              // float4 groups in the tile
     const int f_begin = static_cast<int>(rank) * F / split;
     const int f_end = (static_cast<int>(rank) + 1) * F / split;
     const int qt = static_cast<int>(threadIdx.x) - 64;
@@ -517,14 +527,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < kPer; ++t) {
         const int f = f_begin + qt + t * kQThreads;
         const int m = f / (kBN / 4), n = n0 + (f % (kBN / 4)) * 4;
-        if (f < f_end && m < p.M && n < p.N) {   // N % 8 == 0: a group of 4 is all in or all out
+        if (f < f_end && m < m_end && n < p.N) {   // N % 8 == 0: a group of 4 is all in or all out
+          const int64_t row = m0 + m;
           if (kBf16Out) {
             __nv_bfloat162 lo = __floats2bfloat162_rn(acc[t].x, acc[t].y);
             __nv_bfloat162 hi = __floats2bfloat162_rn(acc[t].z, acc[t].w);
-            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(m) * p.N + n) =
+            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.y) + row * p.N + n) =
                 make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
           } else {
-            *reinterpret_cast<float4*>(static_cast<float*>(p.y) + static_cast<int64_t>(m) * p.N + n) = acc[t];
+            *reinterpret_cast<float4*>(static_cast<float*>(p.y) + row * p.N + n) = acc[t];
           }
         }
       }
@@ -645,6 +656,7 @@ cudaError_t launch_linear_fused(const void* x, int64_t M, int64_t K, const void*
   if (p.group > 3) p.group = 3;   // <= the stages of either layout
   p.idesc_n = static_cast<uint32_t>(p.Mp >> 3) << 17;
   p.act_bytes = 0;
+  p.row_blocks = 1;
   p.skip_fill = -1;
   maps.qx = maps.qr = maps.w;   // unused without kPreQ
   maps.sx = maps.sr = maps.sw;
@@ -660,14 +672,20 @@ cudaError_t launch_gemm_short(const void* qx_codes, const void* qx_scales, const
   EncodeTiledFn encode = reinterpret_cast<EncodeTiledFn>(encode_tiled);
   const bool residual = qr_codes != nullptr;
   const int64_t Mp = (M + 15) / 16 * 16;
-  const uint32_t row_tiles = static_cast<uint32_t>((Mp + 127) / 128);
+  // Above 128 rows, X is taken in blocks of 128 rows, each block a grid row of its own
+  // (2 per weight tile): a CTA's partial tile, and so the split-K exchange through
+  // distributed shared memory, covers 128 rows instead of up to 256 (M = 256, K = N =
+  // 4096, layer after layer: 14.1 against 17.8 us with one 256-row block per CTA).
+  const bool row_split = Mp > 128;
+  const uint32_t box_rows = row_split ? 128u : static_cast<uint32_t>(Mp);
+  const uint32_t row_tiles = row_split ? 1u : static_cast<uint32_t>((Mp + 127) / 128);
   FusedMaps maps;
   if (!encode_codes_map(encode, &maps.w, qw_codes, N, K, kBN)) return cudaErrorInvalidValue;
   if (!encode_scales_map(encode, &maps.sw, qw_scales, N, K, 1)) return cudaErrorInvalidValue;
-  if (!encode_codes_map(encode, &maps.qx, qx_codes, M, K, static_cast<uint32_t>(Mp))) return cudaErrorInvalidValue;
+  if (!encode_codes_map(encode, &maps.qx, qx_codes, M, K, box_rows)) return cudaErrorInvalidValue;
   if (!encode_scales_map(encode, &maps.sx, qx_scales, M, K, row_tiles)) return cudaErrorInvalidValue;
   if (residual) {
-    if (!encode_codes_map(encode, &maps.qr, qr_codes, M, K, static_cast<uint32_t>(Mp))) return cudaErrorInvalidValue;
+    if (!encode_codes_map(encode, &maps.qr, qr_codes, M, K, box_rows)) return cudaErrorInvalidValue;
     if (!encode_scales_map(encode, &maps.sr, qr_scales, M, K, row_tiles)) return cudaErrorInvalidValue;
   } else {
     maps.qr = maps.qx;
@@ -684,13 +702,14 @@ cudaError_t launch_gemm_short(const void* qx_codes, const void* qx_scales, const
   p.num_kt = static_cast<int>((K + kBK - 1) / kBK);
   p.group = 1;
   p.idesc_n = static_cast<uint32_t>(p.Mp >> 3) << 17;
-  // per stage: Mp rows x 128 B of codes and row_tiles x 2 k-atoms of scales, per term
-  p.act_bytes = (static_cast<uint32_t>(Mp) * kBKBytes + row_tiles * 1024u) * (residual ? 2u : 1u);
+  // per stage: a box of rows x 128 B of codes and row_tiles x 2 k-atoms of scales, per term
+  p.act_bytes = (box_rows * kBKBytes + row_tiles * 1024u) * (residual ? 2u : 1u);
+  p.row_blocks = row_split ? 2 : 1;
   p.skip_fill = skip_fill;
-  const int tiles = static_cast<int>((N + kBN - 1) / kBN);
+  const int tiles = static_cast<int>((N + kBN - 1) / kBN) * p.row_blocks;
   // Up to 64 rows: four stages of 43 KiB (measured 10.3 against 11.5 us per layer
-  // at M = 64, K = N = 4096, with the two-stage 85 KiB layout, before the terms were
-  // stacked); up to 128 rows four of 51 KiB; up to 256 two.
+  // at M = 64, K = N = 4096, with a two-stage 85 KiB layout, before the terms were
+  // stacked); otherwise four of 51 KiB per block of 128 rows.
   if (Mp <= 64) {
     if (residual)
       return y_bf16 ? launch_typed<64, true, true, true>(maps, p, tiles, num_sms, stream)
@@ -698,18 +717,11 @@ cudaError_t launch_gemm_short(const void* qx_codes, const void* qx_scales, const
     return y_bf16 ? launch_typed<64, false, true, true>(maps, p, tiles, num_sms, stream)
                   : launch_typed<64, false, false, true>(maps, p, tiles, num_sms, stream);
   }
-  if (Mp <= 128) {
-    if (residual)
-      return y_bf16 ? launch_typed<128, true, true, true>(maps, p, tiles, num_sms, stream)
-                    : launch_typed<128, true, false, true>(maps, p, tiles, num_sms, stream);
-    return y_bf16 ? launch_typed<128, false, true, true>(maps, p, tiles, num_sms, stream)
-                  : launch_typed<128, false, false, true>(maps, p, tiles, num_sms, stream);
-  }
   if (residual)
-    return y_bf16 ? launch_typed<256, true, true, true>(maps, p, tiles, num_sms, stream)
-                  : launch_typed<256, true, false, true>(maps, p, tiles, num_sms, stream);
-  return y_bf16 ? launch_typed<256, false, true, true>(maps, p, tiles, num_sms, stream)
-                : launch_typed<256, false, false, true>(maps, p, tiles, num_sms, stream);
+    return y_bf16 ? launch_typed<128, true, true, true>(maps, p, tiles, num_sms, stream)
+                  : launch_typed<128, true, false, true>(maps, p, tiles, num_sms, stream);
+  return y_bf16 ? launch_typed<128, false, true, true>(maps, p, tiles, num_sms, stream)
+                : launch_typed<128, false, false, true>(maps, p, tiles, num_sms, stream);
 }
 
 void set_fused_split_override(int split) { g_split_override.store(split < 0 ? 0 : split); }

@@ -91,8 +91,8 @@ def test_weight_quantizer_guards(rfq, oracle):
 # (M, N, K): (100, 19200, 256) single-CTA tiled kernel with many tiles; (300, 520, 1024)
 # CTA pairs with ragged M and N (the epilogue's guarded row and column stores);
 # (40, 384, 2304), (96, 520, 2304) and (200, 264, 2304) the short-batch split-K
-# kernel in its three layouts (ragged reduction slices); (1000, 72, 256) a single
-# ragged column tile.
+# kernel at 64 rows, 128 rows and two 128-row blocks (ragged reduction slices and a
+# ragged second block); (1000, 72, 256) a single ragged column tile.
 @pytest.mark.parametrize("M,N,K", [(100, 19200, 256), (300, 520, 1024), (40, 384, 2304), (96, 520, 2304),
                                    (200, 264, 2304), (1000, 72, 256)])
 @pytest.mark.parametrize("residual", [True, False])

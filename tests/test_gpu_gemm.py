@@ -120,9 +120,9 @@ def test_k_zero_writes_zeros(rfq):
 def test_short_batch_gemm_every_split(rfq, oracle, split, M):
     """rfq_gemm on a short batch with few tiles runs the split-K kernel on the
     quantizer's operands: each cluster size (9 k-tiles over 1..8 CTAs, ragged
-    ranges), the three layouts (up to 64 and up to 128 rows with Q(R) stacked under
-    Q(X) in one B operand; up to 256 rows, two 128-row scale atoms of the activation,
-    separate MMAs), bit-identical repeats."""
+    ranges), the layouts (up to 64 and up to 128 rows with Q(R) stacked under Q(X)
+    in one B operand; above 128 rows two 128-row blocks of X on two grid rows per
+    weight tile, the second one ragged), bit-identical repeats."""
     import torch
     N, K = 384, 2304
     x = wl.random_matrix(M, K, seed=M + split, scale=3.0)
