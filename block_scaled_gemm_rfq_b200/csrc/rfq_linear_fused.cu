@@ -135,7 +135,8 @@ struct FusedParams {
   int group;           // k-tiles quantized per round
   uint32_t idesc_n;    // (Mp / 8) << 17
   uint32_t act_bytes;  // kPreQ: bytes of Q(X) [+ Q(R)] codes and scale atoms per stage
-  int row_blocks;      // blocks of kCap rows of X, each a grid row of its own (kPreQ, 128 < M <= 256: 2)
+  int row_blocks;      // blocks of X's rows, each a grid row of its own (1 unless kPreQ and M > block_rows)
+  int block_rows;      // rows per block: 64 or 128 (a multiple of 64: a block lies inside one scale atom)
   int skip_fill;       // kPreQ fault injection: CTA (0, 0) skips this stage fill (-1 = off)
 };
 
@@ -187,12 +188,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_cta_rank();                   // = blockIdx.x
   // Grid rows: weight tiles x row blocks of X (row block fastest, so the clusters of
   // neighbouring rows share the weight tile in L2).  This CTA's rows of X: [m0, m0 + mp),
-  // mp a multiple of 16; rows at and past M (m_end) are zero-filled and not stored.
+  // mp a multiple of 16; rows at and past M (m_end) are zero-filled and not stored.  A
+  // block lies inside one 128-row scale atom (row tile rt); its rows go to the B rows
+  // they have in that atom (from boff = m0 % 128), so that the atom, copied whole to TMEM,
+  // lines up with them: B rows [0, boff) are never read back.
   const int rb = static_cast<int>(blockIdx.y) % p.row_blocks;
   const int tile = static_cast<int>(blockIdx.y) / p.row_blocks;
-  const int m0 = rb * kCap;
-  const int mp = min(p.Mp - m0, kCap);
+  const int m0 = rb * p.block_rows;
+  const int mp = min(p.Mp - m0, p.block_rows);
   const int m_end = p.M - m0;
+  const int rt = m0 >> 7;
+  const int boff = m0 & 127;
   const int n0 = tile * kBN;
   const int kt0 = static_cast<int>(rank) * p.num_kt / split;
   const int nk = (static_cast<int>(rank) + 1) * p.num_kt / split - kt0;   // >= 1: split <= num_kt
@@ -212,11 +218,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (i == p.skip_fill && blockIdx.x == 0 && blockIdx.y == 0) return;   // fault injection (tests)
       // weight tile and the activation's codes and scale atoms, all on one barrier
       mbar_arrive_expect_tx(&wfull[stage], kBN * kBKBytes + 1024u + p.act_bytes);
-      tma_load_2d(st + L::kOffX, &maps.qx, &wfull[stage], kt * kBKBytes, m0);
-      tma_load_4d(st + L::kOffSfx, &maps.sx, &wfull[stage], 0, 0, 2 * kt, rb);
+      tma_load_2d(st + L::kOffX + boff * kBKBytes, &maps.qx, &wfull[stage], kt * kBKBytes, m0);
+      tma_load_4d(st + L::kOffSfx, &maps.sx, &wfull[stage], 0, 0, 2 * kt, rt);
       if (kResidual) {
-        tma_load_2d(st + L::kOffR, &maps.qr, &wfull[stage], kt * kBKBytes, m0);
-        tma_load_4d(st + L::kOffSfr, &maps.sr, &wfull[stage], 0, 0, 2 * kt, rb);
+        tma_load_2d(st + L::kOffR + boff * kBKBytes, &maps.qr, &wfull[stage], kt * kBKBytes, m0);
+        tma_load_4d(st + L::kOffSfr, &maps.sr, &wfull[stage], 0, 0, 2 * kt, rt);
       }
     } else {
       mbar_arrive_expect_tx(&xfull[stage], x_bytes);
@@ -298,6 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // -------------------------------------------------------------- MMA issuer
+      const uint32_t idesc_plain = static_cast<uint32_t>((boff + mp) >> 3) << 17;   // N = boff + mp
       bool ok = true;
       for (int i = 0; i < nk; ++i) {
         const int stage = i % kStages;
@@ -325,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint64_t dw = operand_desc(st + L::kOffW);
           const uint64_t dx = operand_desc(st + L::kOffX);
-          const uint32_t idesc_n = static_cast<uint32_t>((kRRow + mp) >> 3) << 17;
+          const uint32_t idesc_n = static_cast<uint32_t>((kRRow + boff + mp) >> 3) << 17;
 #pragma unroll
           for (uint32_t q = 0; q < 4; ++q) {
             const uint32_t id = 2u * (q & 1u), a = q >> 1;
@@ -353,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (uint32_t q = 0; q < 4; ++q) {
           const uint32_t id = 2u * (q & 1u), a = q >> 1;
-          mma_mxf4(tmem, dw + 2u * q, dx + 2u * q, fused_idesc(p.idesc_n, id), (sf + kSfW + 4 * a) | (id << 30),
+          mma_mxf4(tmem, dw + 2u * q, dx + 2u * q, fused_idesc(idesc_plain, id), (sf + kSfW + 4 * a) | (id << 30),
                    (sf + kSfX + 4 * kRT * a) | (id << 30), (i | static_cast<int>(q)) != 0 ? 1u : 0u);
         }
         if (kResidual) {
@@ -361,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (uint32_t q = 0; q < 4; ++q) {
             const uint32_t id = 2u * (q & 1u), a = q >> 1;
-            mma_mxf4(tmem, dw + 2u * q, dr + 2u * q, fused_idesc(p.idesc_n, id), (sf + kSfW + 4 * a) | (id << 30),
+            mma_mxf4(tmem, dw + 2u * q, dr + 2u * q, fused_idesc(idesc_plain, id), (sf + kSfW + 4 * a) | (id << 30),
                      (sf + kSfR + 4 * kRT * a) | (id << 30), 1u);
           }
         }
@@ -461,10 +468,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n = n0 + n_local;
       for (int c = half; c < mp / 8; c += 2) {
         uint32_t v[8];
-        tmem_load_32x32b_x8(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 8 * c, v);
+        tmem_load_32x32b_x8(tmem + (static_cast<uint32_t>(quad * 32) << 16) + boff + 8 * c, v);
         if constexpr (kStack) {   // + the Q(R) term, kRRow columns further
           uint32_t vr[8];
-          tmem_load_32x32b_x8(tmem + (static_cast<uint32_t>(quad * 32) << 16) + kRRow + 8 * c, vr);
+          tmem_load_32x32b_x8(tmem + (static_cast<uint32_t>(quad * 32) << 16) + kRRow + boff + 8 * c, vr);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 8; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) + __uint_as_float(vr[e]));
@@ -657,6 +664,7 @@ cudaError_t launch_linear_fused(const void* x, int64_t M, int64_t K, const void*
   p.idesc_n = static_cast<uint32_t>(p.Mp >> 3) << 17;
   p.act_bytes = 0;
   p.row_blocks = 1;
+  p.block_rows = p.Mp;
   p.skip_fill = -1;
   maps.qx = maps.qr = maps.w;   // unused without kPreQ
   maps.sx = maps.sr = maps.sw;
@@ -672,13 +680,16 @@ cudaError_t launch_gemm_short(const void* qx_codes, const void* qx_scales, const
   EncodeTiledFn encode = reinterpret_cast<EncodeTiledFn>(encode_tiled);
   const bool residual = qr_codes != nullptr;
   const int64_t Mp = (M + 15) / 16 * 16;
-  // Above 128 rows, X is taken in blocks of 128 rows, each block a grid row of its own
-  // (2 per weight tile): a CTA's partial tile, and so the split-K exchange through
-  // distributed shared memory, covers 128 rows instead of up to 256 (M = 256, K = N =
-  // 4096, layer after layer: 14.1 against 17.8 us with one 256-row block per CTA).
-  const bool row_split = Mp > 128;
-  const uint32_t box_rows = row_split ? 128u : static_cast<uint32_t>(Mp);
-  const uint32_t row_tiles = row_split ? 1u : static_cast<uint32_t>((Mp + 127) / 128);
+  // Above kBlock rows, X is taken in blocks of kBlock rows, each block a grid row of its
+  // own: a CTA's partial tile, and so the split-K exchange through distributed shared
+  // memory, covers one block (M = 256, K = N = 4096, layer after layer: 14.1 us with
+  // blocks of 128 rows against 17.8 with one 256-row block per CTA, and 15.8 with blocks
+  // of 64 rows, where the cluster model then drops the K split: the K loop grows more
+  // than the exchange shrinks).
+  constexpr int64_t kBlock = 128;
+  const bool row_split = Mp > kBlock;
+  const uint32_t box_rows = row_split ? static_cast<uint32_t>(kBlock) : static_cast<uint32_t>(Mp);
+  const uint32_t row_tiles = 1u;
   FusedMaps maps;
   if (!encode_codes_map(encode, &maps.w, qw_codes, N, K, kBN)) return cudaErrorInvalidValue;
   if (!encode_scales_map(encode, &maps.sw, qw_scales, N, K, 1)) return cudaErrorInvalidValue;
@@ -704,7 +715,8 @@ cudaError_t launch_gemm_short(const void* qx_codes, const void* qx_scales, const
   p.idesc_n = static_cast<uint32_t>(p.Mp >> 3) << 17;
   // per stage: a box of rows x 128 B of codes and row_tiles x 2 k-atoms of scales, per term
   p.act_bytes = (box_rows * kBKBytes + row_tiles * 1024u) * (residual ? 2u : 1u);
-  p.row_blocks = row_split ? 2 : 1;
+  p.row_blocks = row_split ? static_cast<int>((Mp + kBlock - 1) / kBlock) : 1;
+  p.block_rows = row_split ? static_cast<int>(kBlock) : static_cast<int>(Mp);
   p.skip_fill = skip_fill;
   const int tiles = static_cast<int>((N + kBN - 1) / kBN) * p.row_blocks;
   // Up to 64 rows: four stages of 43 KiB (measured 10.3 against 11.5 us per layer
