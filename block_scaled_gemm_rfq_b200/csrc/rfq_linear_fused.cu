@@ -78,38 +78,40 @@ constexpr unsigned int kErrWaitQuantX = 7;   // a quantizer warp waiting for its
 //     is 43 KiB (35 without the residual), with 128 rows 51 KiB; four in flight.
 template <int kCap, bool kPreQ, bool kResidual>
 struct FusedLayout {
-  static constexpr int kRowTiles = (kCap + 127) / 128;               // 128-row scale atoms of the activation
-  // Up to 128 rows the Q(R) rows are stacked under the Q(X) rows in one B operand
-  // of kRRow + Mp rows, Q(R) from B row kRRow (a whole number of 8-row swizzle
-  // groups): kCap when the quantizer warps build both terms' scales as one atom;
-  // 128 with pre-quantized operands, so that Q(R)'s own scale atom is copied to
-  // TMEM 4 columns after Q(X)'s (a tcgen05.cp 32x128b destination must start on
-  // a multiple of 4 columns); B rows [Mp, kRRow) are never read back.
-  static constexpr bool kStack = kResidual && kCap <= 128;
-  static constexpr int kRRow = kStack && kPreQ ? 128 : kCap;
-  static constexpr int kStages = kPreQ ? (kCap <= 128 ? 4 : 2) : (kCap <= 32 ? 4 : 3);
+  static_assert(kCap <= 128, "one 128-row scale atom per term and k-atom");
+  // With the residual, Q(R)'s rows are stacked under Q(X)'s in one B operand, Q(R)
+  // from B row kRRow (a whole number of 8-row swizzle groups): kCap when the quantizer
+  // warps build both terms' scales as one atom; 128 with pre-quantized operands, so
+  // that Q(R)'s own scale atom is copied to TMEM 4 columns after Q(X)'s (a tcgen05.cp
+  // 32x128b destination must start on a multiple of 4 columns).  B rows between the
+  // two terms are never read back.
+  static constexpr int kRRow = kPreQ ? 128 : kCap;
+  static constexpr int kXRows = kResidual ? kRRow : kCap;            // B rows before Q(R)'s
+  static constexpr int kStages = kPreQ ? 4 : (kCap <= 32 ? 4 : 3);
   static constexpr uint32_t kBoxBytes = kPreQ ? 0 : kCap * 128;      // one staged box: kCap rows x 64 bf16
   static constexpr uint32_t kOffW = 0;                               // 128 x 128 B of weight codes
   static constexpr uint32_t kOffXs = kOffW + kBN * kBKBytes;         // staged X: 4 boxes (kPreQ: none)
   static constexpr uint32_t kOffX = kOffXs + 4 * kBoxBytes;          // Q(X) codes: kCap x 128 B
-  static constexpr uint32_t kOffR = kOffX + kRRow * kBKBytes;        // Q(R) codes
-  static constexpr uint32_t kOffSfw = kOffR + kCap * kBKBytes;       // 2 k-atoms of 512 B
-  static constexpr uint32_t kOffSfx = kOffSfw + 1024;                // [row tile][k-atom] atoms of 512 B
-  static constexpr uint32_t kOffSfr = kOffSfx + 1024 * kRowTiles;
-  static constexpr uint32_t kStage = kOffSfr + 1024 * kRowTiles;
+  static constexpr uint32_t kOffR = kOffX + kXRows * kBKBytes;       // Q(R) codes (residual kernels)
+  static constexpr uint32_t kOffSfw = kOffR + (kResidual ? kCap : 0) * kBKBytes;   // 2 k-atoms of 512 B
+  static constexpr uint32_t kOffSfx = kOffSfw + 1024;                // the activation's 128-row atom, 2 k-atoms
+  static constexpr uint32_t kOffSfr = kOffSfx + 1024;                // Q(R)'s (pre-quantized residual)
+  static constexpr uint32_t kStage = kOffSfr + 1024;
   // The split-K partial tile ([kCap][128] fp32) reuses stage 0's staged X, or,
   // with kPreQ, the ring: both are dead once the accumulator is complete.
   static constexpr uint32_t kOffRed = kPreQ ? 0 : kOffXs;
   static constexpr uint32_t kOffBar = kStages * kStage;
-  static constexpr uint32_t kSmem = kOffBar + 256 + 1024;
-  // Tensor memory: the accumulator in columns [0, Mp) (stacked terms: [0, kRRow +
-  // Mp)), then one scale slot per stage: +0 QW (2 k-atoms x 4 columns), +kSfX QX
-  // and +kSfR QR (2 k-atoms x kRowTiles x 4 columns each; k-atom a, row tile t at
-  // (a * kRowTiles + t) * 4), or, stacked, both terms' B scales of k-atom a from
-  // +kSfX + 8a.
+  // At least 120 KiB, so that one CTA runs per SM: two co-resident CTAs would share the
+  // SM's tensor core and TMA unit while the split model counts them as two SMs (the
+  // 27 KiB stages of the 64-row kernel without the residual allowed two, and the model
+  // then picked twice the split: 14.2 instead of 8.8 us per layer at M = 64).
+  static constexpr uint32_t kSmem = kOffBar + 256 + 1024 > 120u * 1024u ? kOffBar + 256 + 1024 : 120u * 1024u;
+  // Tensor memory: the accumulator in columns [0, N) (N = B rows, at most kRRow +
+  // kCap), then one scale slot per stage: +0 QW (2 k-atoms x 4 columns), and the B
+  // scales of k-atom a from +kSfX + 8a (4 columns per 128 B rows).
   static constexpr uint32_t kSfBase = kPreQ ? 256 : 128;
   static constexpr uint32_t kSfSlot = kPreQ ? 64 : 32;
-  static constexpr uint32_t kSfW = 0, kSfX = 8, kSfR = 8 + 8 * kRowTiles;
+  static constexpr uint32_t kSfW = 0, kSfX = 8;
   static constexpr uint32_t kTmemCols = kPreQ ? 512 : 256;
   // Per thread and round: blocks (kCap rows x 8 blocks of one stage, or two
   // stages of 16 rows) over kQThreads threads.
@@ -117,9 +119,9 @@ struct FusedLayout {
   static_assert(kOffRed + kCap * kBN * 4 <= (kPreQ ? kStages * kStage : kStage), "partial tile must fit");
   static_assert(kStage % 1024 == 0 && kBoxBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
   static_assert(kSmem <= 232448, "exceeds the 227 KiB shared-memory limit");
-  static_assert(kSfR + 8 * kRowTiles <= kSfSlot, "scale slot too small");
-  // the accumulator: Mp <= kCap columns, or kRRow + Mp with the two terms stacked
-  static_assert(kSfBase >= (kStack ? kRRow + kCap : kCap) && kSfBase + kStages * kSfSlot <= kTmemCols,
+  static_assert(kSfX + 16 <= kSfSlot, "scale slot too small");
+  static_assert(kSfBase >= static_cast<uint32_t>(kXRows + (kResidual ? kCap : 0)) &&
+                    kSfBase + kStages * kSfSlot <= kTmemCols,
                 "scale slots exceed TMEM");
   static_assert((4 * kStages + 2) * 8 + 8 <= 256, "barrier area too small");
 };
@@ -133,7 +135,6 @@ struct FusedParams {
   int Mp;              // MMA N: M rounded up to 16
   int num_kt;          // k-tiles of 256
   int group;           // k-tiles quantized per round
-  uint32_t idesc_n;    // (Mp / 8) << 17
   uint32_t act_bytes;  // kPreQ: bytes of Q(X) [+ Q(R)] codes and scale atoms per stage
   int row_blocks;      // blocks of X's rows, each a grid row of its own (1 unless kPreQ and M > block_rows)
   int block_rows;      // rows per block: 64 or 128 (a multiple of 64: a block lies inside one scale atom)
@@ -168,7 +169,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     rfq_linear_fused_kernel(const __grid_constant__ FusedMaps maps, const FusedParams p) {
   using L = FusedLayout<kCap, kPreQ, kResidual>;
   constexpr int kStages = L::kStages;
-  constexpr bool kStack = L::kStack;
   constexpr int kRRow = L::kRRow;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -304,7 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // -------------------------------------------------------------- MMA issuer
-      const uint32_t idesc_plain = static_cast<uint32_t>((boff + mp) >> 3) << 17;   // N = boff + mp
+      // N = the B rows: Q(X)'s [boff, boff + mp) and, with the residual, Q(R)'s from kRRow + boff
+      const uint32_t idesc_n = static_cast<uint32_t>(((kResidual ? kRRow : 0) + boff + mp) >> 3) << 17;
       bool ok = true;
       for (int i = 0; i < nk; ++i) {
         const int stage = i % kStages;
@@ -317,60 +318,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint8_t* st = smem + stage * L::kStage;
         const uint32_t sf = tmem + L::kSfBase + stage * L::kSfSlot;
-        constexpr uint32_t kSfW = L::kSfW, kSfX = L::kSfX, kSfR = L::kSfR, kRT = L::kRowTiles;
-        if constexpr (kStack) {
-          // B scales of k-atom a from column sf + kSfX + 8a: column c holds B rows
-          // 32c .. 32c + 31.  The quantizer warps write both terms' bytes into one
-          // atom (Q(R)'s at rows kRRow = kCap ..); pre-quantized, Q(R)'s own atom goes
-          // to the 4 columns after Q(X)'s (B rows 128 .. 255).
-#pragma unroll
-          for (uint32_t a = 0; a < 2; ++a) {
-            tmem_copy_32x128b_warpx4_g<1>(sf + kSfW + 4 * a, scale_desc(st + L::kOffSfw + 512 * a));
-            tmem_copy_32x128b_warpx4_g<1>(sf + kSfX + 8 * a, scale_desc(st + L::kOffSfx + 512 * a));
-            if constexpr (kPreQ)
-              tmem_copy_32x128b_warpx4_g<1>(sf + kSfX + 8 * a + 4, scale_desc(st + L::kOffSfr + 512 * a));
-          }
-          const uint64_t dw = operand_desc(st + L::kOffW);
-          const uint64_t dx = operand_desc(st + L::kOffX);
-          const uint32_t idesc_n = static_cast<uint32_t>((kRRow + boff + mp) >> 3) << 17;
-#pragma unroll
-          for (uint32_t q = 0; q < 4; ++q) {
-            const uint32_t id = 2u * (q & 1u), a = q >> 1;
-            mma_mxf4(tmem, dw + 2u * q, dx + 2u * q, fused_idesc(idesc_n, id), (sf + kSfW + 4 * a) | (id << 30),
-                     (sf + kSfX + 8 * a) | (id << 30), (i | static_cast<int>(q)) != 0 ? 1u : 0u);
-          }
-          tc_commit(&empty[stage]);
-          continue;
-        }
+        constexpr uint32_t kSfW = L::kSfW, kSfX = L::kSfX;
+        // Scales: the weight's 2 atoms, and the B scales of k-atom a from column sf +
+        // kSfX + 8a (column c holds B rows 32c .. 32c + 31): Q(X)'s atom, and with the
+        // residual either the same atom (the quantizer warps write Q(R)'s bytes at rows
+        // kRRow = kCap ..) or Q(R)'s own atom 4 columns further (B rows 128 .. 255).
 #pragma unroll
         for (uint32_t a = 0; a < 2; ++a) {
           tmem_copy_32x128b_warpx4_g<1>(sf + kSfW + 4 * a, scale_desc(st + L::kOffSfw + 512 * a));
-#pragma unroll
-          for (uint32_t t = 0; t < kRT; ++t) {
-            // smem atom (row tile t, k-atom a) at (2t + a) * 512 -> columns (a * kRT + t) * 4
-            tmem_copy_32x128b_warpx4_g<1>(sf + kSfX + 4 * (a * kRT + t), scale_desc(st + L::kOffSfx + 512 * (2 * t + a)));
-            if (kResidual)
-              tmem_copy_32x128b_warpx4_g<1>(sf + kSfR + 4 * (a * kRT + t),
-                                            scale_desc(st + L::kOffSfr + 512 * (2 * t + a)));
-          }
+          tmem_copy_32x128b_warpx4_g<1>(sf + kSfX + 8 * a, scale_desc(st + L::kOffSfx + 512 * a));
+          if constexpr (kResidual && kPreQ)
+            tmem_copy_32x128b_warpx4_g<1>(sf + kSfX + 8 * a + 4, scale_desc(st + L::kOffSfr + 512 * a));
         }
         const uint64_t dw = operand_desc(st + L::kOffW);
         const uint64_t dx = operand_desc(st + L::kOffX);
-        // 4 MMAs of K = 64 per term: step q uses k-atom q/2 and scale bytes 2(q%2), 2(q%2)+1.
+        // 4 MMAs of K = 64: step q uses k-atom q/2 and scale bytes 2(q%2), 2(q%2)+1.
 #pragma unroll
         for (uint32_t q = 0; q < 4; ++q) {
           const uint32_t id = 2u * (q & 1u), a = q >> 1;
-          mma_mxf4(tmem, dw + 2u * q, dx + 2u * q, fused_idesc(idesc_plain, id), (sf + kSfW + 4 * a) | (id << 30),
-                   (sf + kSfX + 4 * kRT * a) | (id << 30), (i | static_cast<int>(q)) != 0 ? 1u : 0u);
-        }
-        if (kResidual) {
-          const uint64_t dr = operand_desc(st + L::kOffR);
-#pragma unroll
-          for (uint32_t q = 0; q < 4; ++q) {
-            const uint32_t id = 2u * (q & 1u), a = q >> 1;
-            mma_mxf4(tmem, dw + 2u * q, dr + 2u * q, fused_idesc(idesc_plain, id), (sf + kSfW + 4 * a) | (id << 30),
-                     (sf + kSfR + 4 * kRT * a) | (id << 30), 1u);
-          }
+          mma_mxf4(tmem, dw + 2u * q, dx + 2u * q, fused_idesc(idesc_n, id), (sf + kSfW + 4 * a) | (id << 30),
+                   (sf + kSfX + 8 * a) | (id << 30), (i | static_cast<int>(q)) != 0 ? 1u : 0u);
         }
         tc_commit(&empty[stage]);
       }
@@ -438,13 +405,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(st + L::kOffX + code_off) = make_uint4(cx[0], cx[1], cx[2], cx[3]);
           st[L::kOffSfx + sf_off] = static_cast<uint8_t>(sx);
           if constexpr (kResidual) {
+            // Q(R): B row kRRow + row of the stacked operand, its scale byte in the same atom
             *reinterpret_cast<uint4*>(st + L::kOffR + code_off) = make_uint4(cr[0], cr[1], cr[2], cr[3]);
-            if constexpr (kStack) {   // B row kRRow + row of the stacked operand, same atom
-              const int rr = kRRow + row;
-              st[L::kOffSfx + (j >> 2) * 512u + (rr & 31) * 16u + (rr >> 5) * 4u + (j & 3)] = static_cast<uint8_t>(sr);
-            } else {
-              st[L::kOffSfr + sf_off] = static_cast<uint8_t>(sr);
-            }
+            const int rr = kRRow + row;
+            st[L::kOffSfx + (j >> 2) * 512u + (rr & 31) * 16u + (rr >> 5) * 4u + (j & 3)] = static_cast<uint8_t>(sr);
           }
         }
       }
@@ -469,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = half; c < mp / 8; c += 2) {
         uint32_t v[8];
         tmem_load_32x32b_x8(tmem + (static_cast<uint32_t>(quad * 32) << 16) + boff + 8 * c, v);
-        if constexpr (kStack) {   // + the Q(R) term, kRRow columns further
+        if constexpr (kResidual) {   // + the Q(R) term, kRRow columns further
           uint32_t vr[8];
           tmem_load_32x32b_x8(tmem + (static_cast<uint32_t>(quad * 32) << 16) + kRRow + boff + 8 * c, vr);
           tmem_wait_ld();
@@ -661,7 +625,6 @@ cudaError_t launch_linear_fused(const void* x, int64_t M, int64_t K, const void*
   // Rounds cover kQThreads blocks per slot: two k-tiles at a time for 16 rows.
   p.group = p.Mp * 8 >= kQThreads ? 1 : kQThreads / (p.Mp * 8);
   if (p.group > 3) p.group = 3;   // <= the stages of either layout
-  p.idesc_n = static_cast<uint32_t>(p.Mp >> 3) << 17;
   p.act_bytes = 0;
   p.row_blocks = 1;
   p.block_rows = p.Mp;
@@ -712,7 +675,6 @@ cudaError_t launch_gemm_short(const void* qx_codes, const void* qx_scales, const
   p.Mp = static_cast<int>(Mp);
   p.num_kt = static_cast<int>((K + kBK - 1) / kBK);
   p.group = 1;
-  p.idesc_n = static_cast<uint32_t>(p.Mp >> 3) << 17;
   // per stage: a box of rows x 128 B of codes and row_tiles x 2 k-atoms of scales, per term
   p.act_bytes = (box_rows * kBKBytes + row_tiles * 1024u) * (residual ? 2u : 1u);
   p.row_blocks = row_split ? static_cast<int>((Mp + kBlock - 1) / kBlock) : 1;
