@@ -124,9 +124,11 @@ rfq_status_t rfq_quantize_weight(const void* w_bf16, int64_t N, int64_t K,
  * K multiple of 32; N multiple of 8.  M == 0 or N == 0 launches nothing;
  * K == 0 writes zeros.  Tensor cores: tcgen05 kind::mxf4 block-scaled MMAs.
  * Short batches (M <= 256) whose output tiles would occupy less than half the
- * SMs run a split-K kernel instead: 128 weight rows per CTA, K split over a
- * cluster of up to 8 CTAs, partial sums added in a fixed order (the result
- * differs from the tiled kernel's only by fp32 summation order).
+ * SMs run a split-K kernel instead: 128 weight rows and up to 128 rows of X per
+ * CTA (two row blocks above 128 rows), K split over a cluster of up to 8 CTAs,
+ * the Q(X) and Q(R) products in separate accumulator columns added per output,
+ * partial sums added in a fixed order (the result differs from the tiled
+ * kernel's only by fp32 summation order).
  */
 rfq_status_t rfq_gemm(const void* qx_codes, const void* qx_scales,
                       const void* qr_codes, const void* qr_scales,
@@ -367,9 +369,10 @@ rfq_status_t rfq_check_device_error(cudaStream_t stream, int* detail);
 rfq_status_t rfq_debug_skip_next_fill(int fill_index);
 
 /*
- * Tuning hook: make rfq_linear_fused split K over `split` CTAs (1..8, capped at
- * the number of 256-element k-tiles) instead of choosing from the device's
- * occupancy; 0 restores the automatic choice.  Process-wide.
+ * Tuning hook: make rfq_linear_fused and the short-batch path of rfq_gemm split
+ * K over `split` CTAs (1..8, capped at the number of 256-element k-tiles)
+ * instead of choosing from the device's occupancy; 0 restores the automatic
+ * choice.  Process-wide.
  */
 rfq_status_t rfq_debug_fused_split(int split);
 
