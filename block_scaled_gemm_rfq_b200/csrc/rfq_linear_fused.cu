@@ -61,9 +61,16 @@ namespace {
 constexpr int kBN = 128;                  // weight rows per tile = MMA M = columns of Y per tile
 constexpr int kBK = 256;                  // K per stage
 constexpr int kBKBytes = kBK / 2;         // 128 bytes of codes per row per stage
-constexpr int kQWarps = 8;                // quantizer warps, then epilogue warps
-constexpr int kQThreads = kQWarps * 32;
-constexpr int kThreads = 64 + kQThreads;  // warp 0 TMA, warp 1 MMA, warps 2..9 quantize + epilogue
+// Warps 2 .. 2 + kQW quantize (bf16 input) and then run the epilogue: 16 of them for
+// 17-32 rows, 8 otherwise, so that a quantization round covers two k-tiles with one
+// block per thread for 16 and for 32 rows.  (Rounds of one k-tile for 32 rows: 9.2 us
+// per layer at M = 32 against 8.8; one round of four k-tiles for 16 rows: 8.1 against
+// 7.1 us, the MMAs waiting for all four stages of X.)  Warp 0 issues TMA, warp 1 MMAs.
+template <int kQW>
+struct FusedWarps {
+  static constexpr int kQT = kQW * 32;
+  static constexpr int kThreads = 64 + kQT;
+};
 constexpr int kMaxSplit = 8;              // portable cluster size
 constexpr int kMaxDevices = 64;
 constexpr unsigned int kErrWaitQuantX = 7;   // a quantizer warp waiting for its staged X
@@ -76,7 +83,7 @@ constexpr unsigned int kErrWaitQuantX = 7;   // a quantizer warp waiting for its
 //     short-batch GEMM: 32 < M <= 256, or any rfq_gemm call with few tiles; above
 //     128 rows each CTA takes one 128-row block of X); with up to 64 rows a stage
 //     is 43 KiB (35 without the residual), with 128 rows 51 KiB; four in flight.
-template <int kCap, bool kPreQ, bool kResidual>
+template <int kCap, bool kPreQ, bool kResidual, int kQW = 8>
 struct FusedLayout {
   static_assert(kCap <= 128, "one 128-row scale atom per term and k-atom");
   // With the residual, Q(R)'s rows are stacked under Q(X)'s in one B operand, Q(R)
@@ -113,9 +120,10 @@ struct FusedLayout {
   static constexpr uint32_t kSfSlot = kPreQ ? 64 : 32;
   static constexpr uint32_t kSfW = 0, kSfX = 8;
   static constexpr uint32_t kTmemCols = kPreQ ? 512 : 256;
-  // Per thread and round: blocks (kCap rows x 8 blocks of one stage, or two
-  // stages of 16 rows) over kQThreads threads.
-  static constexpr int kSlots = kCap * 8 / kQThreads > 0 ? kCap * 8 / kQThreads : 1;
+  // Per thread and round: blocks (kCap rows x 8 blocks of one stage, or several
+  // stages of 16 rows) over the quantizer threads.
+  static constexpr int kQT = FusedWarps<kQW>::kQT;
+  static constexpr int kSlots = kCap * 8 / kQT > 0 ? kCap * 8 / kQT : 1;
   static_assert(kOffRed + kCap * kBN * 4 <= (kPreQ ? kStages * kStage : kStage), "partial tile must fit");
   static_assert(kStage % 1024 == 0 && kBoxBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
   static_assert(kSmem <= 232448, "exceeds the 227 KiB shared-memory limit");
@@ -164,11 +172,13 @@ __device__ __forceinline__ uint32_t fused_idesc(uint32_t idesc_n, uint32_t sf_id
   return (sf_id << 4) | (1u << 7) | (1u << 10) | idesc_n | (1u << 23) | (uint32_t(kBN >> 4) << 24) | (sf_id << 29);
 }
 
-template <int kCap, bool kResidual, bool kBf16Out, bool kPreQ>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int kCap, bool kResidual, bool kBf16Out, bool kPreQ, int kQW>
+__global__ void __launch_bounds__(FusedWarps<kQW>::kThreads, 1)
     rfq_linear_fused_kernel(const __grid_constant__ FusedMaps maps, const FusedParams p) {
-  using L = FusedLayout<kCap, kPreQ, kResidual>;
+  using L = FusedLayout<kCap, kPreQ, kResidual, kQW>;
   constexpr int kStages = L::kStages;
+  constexpr int kQWarps = kQW;
+  constexpr int kQThreads = FusedWarps<kQW>::kQT;
   constexpr int kRRow = L::kRRow;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -420,17 +430,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------------------------------------------------------- epilogue
     // Warp w reads TMEM lanes 32 (w % 4) .. +31 (weight rows = columns of Y);
-    // the two warps of a lane quadrant alternate over 8-column chunks (rows of X).
+    // the warps of a lane quadrant alternate over 8-column chunks (rows of X).
     // With a K split the accumulator goes, as [Mp][128] fp32, to this CTA's
     // receive area for the cluster reduction below.
     epi_ok = mbar_wait(acc_full, 0, abort_flag, &g_fused_error, kErrWaitAccFull, 2 * kWaitLimitNs);
     if (__all_sync(0xffffffffu, epi_ok)) {
       tc_fence_after();
       const int quad = warp & 3;
-      const int half = (warp - 2) >> 2;
+      const int half = (warp - 2) >> 2;   // the warps of a lane quadrant take turns over 8-column chunks
       const int n_local = quad * 32 + lane;
       const int n = n0 + n_local;
-      for (int c = half; c < mp / 8; c += 2) {
+      for (int c = half; c < mp / 8; c += kQWarps / 4) {
         uint32_t v[8];
         tmem_load_32x32b_x8(tmem + (static_cast<uint32_t>(quad * 32) << 16) + boff + 8 * c, v);
         if constexpr (kResidual) {   // + the Q(R) term, kRRow columns further
@@ -468,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // distributed stores instead measured slower; the exchange is bound by the
     // distributed shared-memory bandwidth either way.)
     cluster_sync();
-    constexpr int kPer = kCap / 16;            // >= ceil(F / split / kQThreads) for split >= 2
+    constexpr int kPer = kCap / 16;            // >= ceil(F / split / kQThreads) for split >= 2 (kQThreads >= 256)
     float4 acc[kPer];
     const int F = mp * (kBN / 4);              // float4 groups in the tile
     const int f_begin = static_cast<int>(rank) * F / split;
@@ -525,16 +535,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 std::atomic<int> g_split_override{0};
 
-template <int kCap, bool kResidual, bool kBf16Out, bool kPreQ = false>
+template <int kCap, bool kResidual, bool kBf16Out, bool kPreQ = false, int kQW = 8>
 cudaError_t launch_typed(const FusedMaps& maps, const FusedParams& p, int tiles, int num_sms, cudaStream_t stream) {
-  using L = FusedLayout<kCap, kPreQ, kResidual>;
-  auto kernel = rfq_linear_fused_kernel<kCap, kResidual, kBf16Out, kPreQ>;
+  using L = FusedLayout<kCap, kPreQ, kResidual, kQW>;
+  auto kernel = rfq_linear_fused_kernel<kCap, kResidual, kBf16Out, kPreQ, kQW>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(FusedWarps<kQW>::kThreads);
   cfg.dynamicSmemBytes = L::kSmem;
   cfg.stream = stream;
+  FusedParams q = p;
+  if constexpr (!kPreQ) {
+    // A quantization round gives each quantizer thread one block: k-tiles of Mp rows x 8
+    // blocks, as many as the threads cover (all four stages of a CTA's range for 16 rows
+    // and 16 warps), at most the ring's stages, which must all hold their staged X at once.
+    constexpr int kQT = FusedWarps<kQW>::kQT;
+    q.group = q.Mp * 8 >= kQT ? 1 : kQT / (q.Mp * 8);
+    if (q.group > L::kStages) q.group = L::kStages;
+  }
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.y = 1;
@@ -578,19 +597,19 @@ cudaError_t launch_typed(const FusedMaps& maps, const FusedParams& p, int tiles,
   if (split > kMaxSplit) split = kMaxSplit;
   attr[0].val.clusterDim.x = split;
   cfg.gridDim = dim3(split, tiles);
-  e = cudaLaunchKernelEx(&cfg, kernel, maps, p);
+  e = cudaLaunchKernelEx(&cfg, kernel, maps, q);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-template <int kCap>
+template <int kCap, int kQW = 8>
 cudaError_t launch_cap(const FusedMaps& maps, const FusedParams& p, int tiles, bool residual, bool y_bf16,
                        int num_sms, cudaStream_t stream) {
   if (residual)
-    return y_bf16 ? launch_typed<kCap, true, true>(maps, p, tiles, num_sms, stream)
-                  : launch_typed<kCap, true, false>(maps, p, tiles, num_sms, stream);
-  return y_bf16 ? launch_typed<kCap, false, true>(maps, p, tiles, num_sms, stream)
-                : launch_typed<kCap, false, false>(maps, p, tiles, num_sms, stream);
+    return y_bf16 ? launch_typed<kCap, true, true, false, kQW>(maps, p, tiles, num_sms, stream)
+                  : launch_typed<kCap, true, false, false, kQW>(maps, p, tiles, num_sms, stream);
+  return y_bf16 ? launch_typed<kCap, false, true, false, kQW>(maps, p, tiles, num_sms, stream)
+                : launch_typed<kCap, false, false, false, kQW>(maps, p, tiles, num_sms, stream);
 }
 
 }  // namespace
@@ -622,9 +641,7 @@ cudaError_t launch_linear_fused(const void* x, int64_t M, int64_t K, const void*
   p.Kb = static_cast<int>(K / 32);
   p.Mp = static_cast<int>(Mp);
   p.num_kt = static_cast<int>((K + kBK - 1) / kBK);
-  // Rounds cover kQThreads blocks per slot: two k-tiles at a time for 16 rows.
-  p.group = p.Mp * 8 >= kQThreads ? 1 : kQThreads / (p.Mp * 8);
-  if (p.group > 3) p.group = 3;   // <= the stages of either layout
+  p.group = 1;   // set per layout in launch_typed
   p.act_bytes = 0;
   p.row_blocks = 1;
   p.block_rows = p.Mp;
@@ -632,8 +649,9 @@ cudaError_t launch_linear_fused(const void* x, int64_t M, int64_t K, const void*
   maps.qx = maps.qr = maps.w;   // unused without kPreQ
   maps.sx = maps.sr = maps.sw;
   const int tiles = static_cast<int>((N + kBN - 1) / kBN);
-  return p.Mp <= 32 ? launch_cap<32>(maps, p, tiles, residual, y_bf16, num_sms, stream)
-                    : launch_cap<64>(maps, p, tiles, residual, y_bf16, num_sms, stream);
+  if (p.Mp <= 16) return launch_cap<32, 8>(maps, p, tiles, residual, y_bf16, num_sms, stream);
+  return p.Mp <= 32 ? launch_cap<32, 16>(maps, p, tiles, residual, y_bf16, num_sms, stream)
+                    : launch_cap<64, 8>(maps, p, tiles, residual, y_bf16, num_sms, stream);
 }
 
 cudaError_t launch_gemm_short(const void* qx_codes, const void* qx_scales, const void* qr_codes,

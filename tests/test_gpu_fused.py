@@ -43,11 +43,13 @@ def test_fused_edge_shapes(rfq, oracle, M, N, K, residual):
 
 
 @pytest.mark.parametrize("split", [1, 2, 3, 5, 8])
-def test_fused_every_split(rfq, oracle, split):
-    """Each cluster size (ragged k-ranges included: 9 k-tiles over 2, 3, 5, 8 CTAs)."""
+@pytest.mark.parametrize("M", [12, 24])
+def test_fused_every_split(rfq, oracle, split, M):
+    """Each cluster size (ragged k-ranges included: 9 k-tiles over 2, 3, 5, 8 CTAs), with
+    8 quantizer warps (up to 16 rows) and with 16 (17-32 rows)."""
     import torch
-    M, N, K = 24, 384, 2304
-    x = wl.random_matrix(M, K, seed=21, scale=3.0)
+    N, K = 384, 2304
+    x = wl.random_matrix(M, K, seed=21 + M, scale=3.0)
     w = wl.random_matrix(N, K, seed=22, scale=0.05)
     Y, S, _ = oracle.rfq_linear(x, w, residual=True)
     for out in (torch.float32, torch.bfloat16):
