@@ -1,5 +1,6 @@
 // rfq_linear_fused.cu -- the RFQ linear layer in one kernel for short batches
-// (M <= 64 rows of X): the quantizer runs in the GEMM's producer warps.
+// (M <= 64 rows of X): the quantizer runs in the GEMM's producer warps; and the
+// same kernel on pre-quantized operands, the short-batch GEMM (M <= 256).
 //
 // "Activation Outliers Matter: Robust Recovery for Quantized Multimodal LLMs",
 // section 1 (RFQ contribution paragraph): X is quantized to FP4, its residual
@@ -22,7 +23,7 @@
 //   * warp 0 streams, per stage, the bf16 rows of X for the k-tile (4 boxes of
 //     Mp rows x 64 elements, 128-byte swizzle; rows past M read as zeros) and
 //     the weight tile with its scale atoms, all with TMA, kStages ahead;
-//   * warps 2..9 quantize each 32-element block of the staged X with the same
+//   * warps 2..9 (2..17 for 17-32 rows) quantize each 32-element block of the staged X with the same
 //     arithmetic as the stand-alone quantizer and write the codes into the
 //     swizzled B-operand tile and the E8M0 bytes into the stage's scale atoms in
 //     shared memory -- Q(X) and Q(R) never reach global memory;
