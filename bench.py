@@ -414,6 +414,26 @@ def time_gemm_pair(rfq, x, w, flush, iters):
             "tflops_executed_rfq": 4.0 * M * N * K / (statistics.mean(t_on) * 1e-3) / 1e12}
 
 
+def concat_scales_along_k(s1, s2, rows: int, K: int):
+    """The E8M0 scale arrays of two [rows][K] MX operands, in the block-scaled MMA layout
+    (atoms of 128 rows x 4 blocks, 512 bytes, the block index fastest: the layout the
+    quantizer writes and cuBLASLt's 32x4x4 swizzle), joined into the scales of the
+    [rows][2K] operand [A1 | A2]: per 128-row tile, A1's K/128 atoms then A2's.  K must be
+    a multiple of 128 (whole atoms).  Works on torch tensors and numpy arrays alike."""
+    if K % 128:
+        raise ValueError("K must be a multiple of 128")
+    rt, kb4 = (rows + 127) // 128, K // 128
+    a, b = s1.reshape(rt, kb4, 512), s2.reshape(rt, kb4, 512)
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            return torch.cat([a, b], dim=1).reshape(-1)
+    except ImportError:
+        pass
+    import numpy as np
+    return np.concatenate([a, b], axis=1).reshape(-1)
+
+
 def time_library_gemm(rfq, step, flush, iters):
     """A library comparator on the step's own quantized operands: cuBLASLt's MXFP4 GEMM
     (torch's scaled_mm, 1x32 E8M0 block scales in the 32x4x4 swizzled layout, which is
@@ -430,16 +450,15 @@ def time_library_gemm(rfq, step, flush, iters):
     M, N, K = step.M, step.N, step.K
     if K % 128:
         return {"unavailable": "K is not a multiple of 128"}
-    Kb, rtx, rtw, kb4 = K // 2, (M + 127) // 128, (N + 127) // 128, K // 128
+    Kb = K // 2
 
     def lib(a, b, sa, sb, kb):
         return F.scaled_mm(a.view(M, kb).view(fp4), b.view(N, kb).view(fp4).t(), sa.view(e8), BW, sb.view(e8), BW,
                            swizzle_a=SW, swizzle_b=SW, output_dtype=torch.bfloat16)
 
-    cat_s = lambda s1, s2, rt: torch.cat([s1.view(rt, kb4, 512), s2.view(rt, kb4, 512)], dim=1).reshape(-1)
     a2 = torch.cat([step.qx_c.view(M, Kb), step.qr_c.view(M, Kb)], dim=1)
     b2 = torch.cat([step.qw_c.view(N, Kb), step.qw_c.view(N, Kb)], dim=1)
-    sa2, sb2 = cat_s(step.qx_s, step.qr_s, rtx), cat_s(step.qw_s, step.qw_s, rtw)
+    sa2, sb2 = concat_scales_along_k(step.qx_s, step.qr_s, M, K), concat_scales_along_k(step.qw_s, step.qw_s, N, K)
     try:
         y_lib = lib(a2, b2, sa2, sb2, 2 * Kb)
     except Exception as e:   # no MXFP4 kernel for this device or build

@@ -11,6 +11,7 @@ path never calls it.  Skipped where torch has no MXFP4 scaled_mm for the device.
 import numpy as np
 import pytest
 
+import bench
 from block_scaled_gemm_rfq_b200 import workloads as wl
 from helpers import REL_TOL, assert_y_close, bf16_ulp, dev_bf16, y_to_numpy
 
@@ -36,13 +37,14 @@ def test_library_gemm_reads_our_operands(rfq, oracle, M, N, K):
     w_bits = wl.random_matrix(N, K, seed=N + 6, scale=0.05)
     qa = rfq.quantize_mxfp4_alloc(dev_bf16(x_bits), residual=True)
     qw = rfq.quantize_weight_alloc(dev_bf16(w_bits))
-    kb, kb4 = K // 2, K // 128
-    cat_s = lambda s1, s2: torch.cat([s1.view(-1, kb4, 512), s2.view(-1, kb4, 512)], dim=1).reshape(-1)
+    kb = K // 2
     a2 = torch.cat([qa.codes.view(M, kb), qa.r_codes.view(M, kb)], dim=1)
     b2 = torch.cat([qw.codes.view(N, kb), qw.codes.view(N, kb)], dim=1)
+    sa2 = bench.concat_scales_along_k(qa.scales, qa.r_scales, M, K)
+    sb2 = bench.concat_scales_along_k(qw.scales, qw.scales, N, K)
     try:
         y_plain = _lib_mm(qa.codes, qw.codes, qa.scales, qw.scales, M, N, kb)
-        y_lib = _lib_mm(a2, b2, cat_s(qa.scales, qa.r_scales), cat_s(qw.scales, qw.scales), M, N, 2 * kb)
+        y_lib = _lib_mm(a2, b2, sa2, sb2, M, N, 2 * kb)
     except (RuntimeError, ValueError) as e:
         pytest.skip(f"no MXFP4 scaled_mm here: {str(e)[:120]}")
     y_ours = rfq.gemm_alloc(qa, qw, out_dtype=torch.bfloat16, use_residual=True)
