@@ -140,3 +140,24 @@ def test_short_batch_gemm_every_split(rfq, oracle, split, M):
     assert_y_close(y_to_numpy(ys[0]), Y, S, bf16_out=False, what=f"short M={M} split {split}")
     assert_y_close(y_to_numpy(ys[1]), Y, S, bf16_out=True, what=f"short M={M} split {split} bf16")
     assert torch.equal(ys[0].view(torch.int32), ys[2].view(torch.int32))
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 4096, 512), (1000, 2056, 768), (200, 1032, 2304), (24, 520, 1024)])
+@pytest.mark.parametrize("residual", [True, False])
+def test_repeat_and_output_types_agree_bitwise(rfq, M, N, K, residual):
+    """Every path (the persistent CTA-pair kernel over several waves, ragged tiles, the
+    short-batch split-K kernel) gives bit-identical Y on a repeat call, and its bf16 Y is
+    exactly the round-to-nearest-even of its fp32 Y: both come from the same fp32
+    accumulation, whatever warp issues the scale copies or the MMAs."""
+    import torch
+    x = wl.random_matrix(M, K, seed=M + K + 1, scale=2.0)
+    w = wl.random_matrix(N, K, seed=N + K + 2, scale=0.05)
+    qa = rfq.quantize_mxfp4_alloc(dev_bf16(x), residual=residual)
+    qw = rfq.quantize_weight_alloc(dev_bf16(w))
+    y32a = rfq.gemm_alloc(qa, qw, out_dtype=torch.float32, use_residual=residual)
+    y32b = rfq.gemm_alloc(qa, qw, out_dtype=torch.float32, use_residual=residual)
+    y16 = rfq.gemm_alloc(qa, qw, out_dtype=torch.bfloat16, use_residual=residual)
+    torch.cuda.synchronize()
+    rfq.check_device_error()
+    assert torch.equal(y32a.view(torch.int32), y32b.view(torch.int32)), "repeat differs"
+    assert torch.equal(y16.view(torch.int16), y32a.to(torch.bfloat16).view(torch.int16)), "bf16 Y != rne(fp32 Y)"
