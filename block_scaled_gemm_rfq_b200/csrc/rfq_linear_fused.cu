@@ -129,6 +129,11 @@ struct FusedLayout {
   static_assert(kStage % 1024 == 0 && kBoxBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
   static_assert(kSmem <= 232448, "exceeds the 227 KiB shared-memory limit");
   static_assert(kSfX + 16 <= kSfSlot, "scale slot too small");
+  // tcgen05.cp 32x128b destinations start on a multiple of 4 TMEM columns
+  static_assert(kSfBase % 4 == 0 && kSfSlot % 4 == 0 && kSfW % 4 == 0 && kSfX % 4 == 0, "scale copy alignment");
+  // the B operand (Q(X) rows, then Q(R)'s from kRRow) is at most N = 256 rows and stays in the stage
+  static_assert((kResidual ? kRRow + kCap : kCap) <= 256, "MMA N exceeds 256");
+  static_assert(kOffX + (kResidual ? kRRow + kCap : kCap) * kBKBytes <= kOffSfw, "B operand leaves its area");
   static_assert(kSfBase >= static_cast<uint32_t>(kXRows + (kResidual ? kCap : 0)) &&
                     kSfBase + kStages * kSfSlot <= kTmemCols,
                 "scale slots exceed TMEM");
