@@ -70,6 +70,8 @@ constexpr uint32_t kSfSlot = 32;
 constexpr uint32_t kSfaXCol = 0;       // +4a..4a+3:   QX, this CTA's 128 rows
 constexpr uint32_t kSfaRCol = 8;       // +8+4a..:     QR
 constexpr uint32_t kSfbCol = 16;       // +16+8a..+7:  QW, the tile's 256 rows (2 row atoms)
+static_assert(kSfBase % 4 == 0 && kSfSlot % 4 == 0 && kSfaXCol % 4 == 0 && kSfaRCol % 4 == 0 && kSfbCol % 4 == 0,
+              "tcgen05.cp 32x128b destinations start on a multiple of 4 TMEM columns");
 constexpr uint32_t kSmemLimit = 232448;
 
 // One ring stage: the QX tile, the QR tile (residual kernels only), this CTA's part
